@@ -1,0 +1,372 @@
+"""Pins for the CPU oracle: each check comes from outside the oracle itself.
+
+* reorder/unorder: explicit closed-form packed index per (t, y, x), zero pad
+  rows, round trip;
+* pooling: closed-form means of constant and linear fields over the valid part
+  of each tile;
+* scores: the identity "dot of tile means = block average of the token Gram
+  matrix" and orthonormal-basis inputs;
+* top-k: brute force over every k-subset (max score sum, lexicographically
+  smallest on ties) with planted ties;
+* window: brute force over every feasible start per axis (the start closest to
+  the centred one) plus the pages' "within +-w/2" interior rule;
+* attention: torch's scaled_dot_product_attention in float64 on the raster
+  tokens with a token-level mask built in raster space (dense, block-diagonal
+  and random kept sets), and torch.logsumexp for LSE.
+
+Sources: "HunyuanVideo 1.5 Technical Report" (paper-graph-ui summary),
+section "SSTA: Selective and Sliding Tile Attention", Steps 1-4 and the
+attention equation.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssta_inputs as si
+from ssta_inputs import Workload, with_overrides
+
+
+def _desc(T=5, Y=6, X=7, tT=2, tY=4, tX=3, wT=1, wY=1, wX=1, topk=2, L_text=0, H=2, D=8, B=1):
+    return Workload("pin", "f32", B, H, D, T, Y, X, tT, tY, tX, wT, wY, wX, topk, L_text,
+                    "tile_offset")
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# Step 1: reorder / unorder
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L_text", [0, 5])
+def test_reorder_closed_form_index(L_text):
+    d = _desc(L_text=L_text)
+    g = oracle.geometry(d)
+    x = _rand((d.B, d.H, d.T, d.Y, d.X, d.D), 1)
+    xt = _rand((d.B, d.H, L_text, d.D), 2) if L_text else None
+    p = oracle.tile_reorder(d, x, xt)
+    assert p.shape == (d.B, d.H, g.NT * g.N + L_text, d.D)
+    nY, nX = -(-d.Y // d.tY), -(-d.X // d.tX)
+    N = d.tT * d.tY * d.tX
+    hit = np.zeros(p.shape[2], dtype=bool)
+    for t in range(d.T):
+        for y in range(d.Y):
+            for xx in range(d.X):
+                c = ((t // d.tT) * nY + y // d.tY) * nX + xx // d.tX
+                o = ((t % d.tT) * d.tY + y % d.tY) * d.tX + xx % d.tX
+                r = c * N + o
+                np.testing.assert_array_equal(p[:, :, r], x[:, :, t, y, xx])
+                hit[r] = True
+    # every other video row is a pad row and holds zeros
+    assert np.all(p[:, :, : g.NT * N][:, :, ~hit[: g.NT * N]] == 0)
+    assert hit[: g.NT * N].sum() == d.T * d.Y * d.X
+    if L_text:
+        np.testing.assert_array_equal(p[:, :, g.NT * N:], xt)
+    np.testing.assert_array_equal(oracle.valid_token_mask(d)[: g.NT * N], hit[: g.NT * N])
+    back, back_t = oracle.tile_unorder(d, p)
+    np.testing.assert_array_equal(back, x)
+    if L_text:
+        np.testing.assert_array_equal(back_t, xt)
+
+
+def test_geometry_of_workloads():
+    # grid sizes of the video latents: tiles after rounding up, top-k clamp
+    expect = {"tiny_f32": (8, 32, 8, 256), "small_bf16": (112, 256, 112, 28672),
+              "p480_5s_bf16": (224, 256, 224, 57344),
+              "p720_5s_bf16": (480, 256, 481, 480 * 256 + 256),
+              "p720_10s_bf16": (960, 256, 961, 960 * 256 + 256)}
+    for name, (NT, N, NQ, Lq) in expect.items():
+        g = oracle.geometry(si.get_workload(name))
+        assert (g.NT, g.N, g.NQ, g.Lq) == (NT, N, NQ, Lq), name
+    assert oracle.geometry(_desc(topk=99)).k == oracle.geometry(_desc()).NT
+
+
+# ---------------------------------------------------------------------------
+# Step 2: pooling, scores, top-k
+# ---------------------------------------------------------------------------
+
+def test_pool_constant_and_linear():
+    d = _desc(D=3)
+    g = oracle.geometry(d)
+    t, y, x = np.meshgrid(np.arange(d.T), np.arange(d.Y), np.arange(d.X), indexing="ij")
+    field = np.stack([np.full(t.shape, 2.5), 3.0 * t - 2.0 * y + 0.5 * x, 7.0 * x], axis=-1)
+    raster = np.broadcast_to(field, (d.B, d.H) + field.shape).copy()
+    pooled = oracle.tile_pool(d, oracle.tile_reorder(d, raster, None))
+    nY, nX = g.nY, g.nX
+    for cT in range(g.nT):
+        for cY in range(nY):
+            for cX in range(nX):
+                c = (cT * nY + cY) * nX + cX
+                # mean of a linear function over a box = value at the box's valid centre
+                def centre(ci, tl, n):
+                    lo, hi = ci * tl, min(ci * tl + tl, n) - 1
+                    return 0.5 * (lo + hi)
+                mt, my, mx = centre(cT, d.tT, d.T), centre(cY, d.tY, d.Y), centre(cX, d.tX, d.X)
+                np.testing.assert_allclose(pooled[0, 1, c], [2.5, 3 * mt - 2 * my + 0.5 * mx, 7 * mx],
+                                           rtol=0, atol=1e-12)
+
+
+def test_scores_equal_block_average_of_token_gram():
+    d = _desc(D=5, T=4, Y=5, X=3)
+    g = oracle.geometry(d)
+    q = _rand((1, 2, d.T, d.Y, d.X, d.D), 3)
+    k = _rand((1, 2, d.T, d.Y, d.X, d.D), 4)
+    S = oracle.tile_scores(d, oracle.tile_pool(d, oracle.tile_reorder(d, q, None)),
+                           oracle.tile_pool(d, oracle.tile_reorder(d, k, None)))
+    # tile membership computed in raster space, token Gram matrix averaged per block pair
+    t, y, x = np.meshgrid(np.arange(d.T), np.arange(d.Y), np.arange(d.X), indexing="ij")
+    member = (((t // d.tT) * g.nY + y // d.tY) * g.nX + x // d.tX).reshape(-1)
+    for h in range(2):
+        G = q[0, h].reshape(-1, d.D) @ k[0, h].reshape(-1, d.D).T
+        for i in range(g.NT):
+            for j in range(g.NT):
+                blk = G[np.ix_(member == i, member == j)]
+                assert abs(blk.mean() - S[0, h, i, j]) < 1e-10
+
+
+def test_scores_orthonormal_basis():
+    d = _desc(D=8, T=2, Y=4, X=6, tT=2, tY=4, tX=3)   # NT = 2 tiles
+    q = np.zeros((1, 1, 2, 4, 6, 8))
+    k = np.zeros_like(q)
+    q[..., :3, 0] = 1.0   # tile 0 -> e0
+    q[..., 3:, 1] = 1.0   # tile 1 -> e1
+    k[..., :3, 1] = 2.0   # tile 0 -> 2 e1
+    k[..., 3:, 0] = -1.0  # tile 1 -> -e0
+    S = oracle.tile_scores(d, oracle.tile_pool(d, oracle.tile_reorder(d, q, None)),
+                           oracle.tile_pool(d, oracle.tile_reorder(d, k, None)))
+    np.testing.assert_array_equal(S[0, 0], [[0.0, -1.0], [2.0, 0.0]])
+
+
+def _brute_topk(scores_row, k):
+    best, best_key = None, None
+    for sub in itertools.combinations(range(len(scores_row)), k):
+        total = float(sum(float(scores_row[j]) for j in sub))
+        key = (-total, sub)
+        if best_key is None or key < best_key:
+            best, best_key = sub, key
+    return set(best)
+
+
+@pytest.mark.parametrize("NT_grid", [(1, 2, 3), (2, 2, 2)])
+def test_topk_brute_force_with_ties(NT_grid):
+    nT, nY, nX = NT_grid
+    d = _desc(T=nT, Y=nY, X=nX, tT=1, tY=1, tX=1)
+    NT = nT * nY * nX
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        # quantised scores -> many exact ties; sums are exact in float64
+        S = (rng.integers(-3, 4, size=(1, 1, NT, NT)) * 0.25).astype(np.float64)
+        if trial % 4 == 0:
+            S = rng.standard_normal((1, 1, NT, NT))
+        for k in range(0, NT + 2):
+            dk = with_overrides(d, topk=k)
+            sel = oracle.select_topk(dk, S)
+            for i in range(NT):
+                want = _brute_topk(S[0, 0, i].astype(np.float32), min(k, NT))
+                assert set(np.nonzero(sel[0, 0, i])[0]) == want, (trial, k, i)
+
+
+def test_topk_decision_in_float32():
+    # two scores that differ only below float32 resolution tie; the lower index wins
+    d = _desc(T=1, Y=1, X=3, tT=1, tY=1, tX=1, topk=1)
+    S = np.array([[[[1.0, 1.0 + 1e-12, 0.5]] * 3]])
+    sel = oracle.select_topk(d, S)
+    assert list(np.nonzero(sel[0, 0, 0])[0]) == [0]
+
+
+# ---------------------------------------------------------------------------
+# Step 3: window
+# ---------------------------------------------------------------------------
+
+def _brute_axis_window(n, w, c):
+    span = min(w, n)
+    starts = range(0, n - span + 1)
+    want = c - w // 2
+    s = min(starts, key=lambda s: (abs(s - want), s))
+    return set(range(s, s + span))
+
+
+@pytest.mark.parametrize("n", range(1, 8))
+@pytest.mark.parametrize("w", range(1, 10))
+def test_axis_window_brute_force(n, w):
+    m = oracle.ssta_oracle._axis_window(n, w)
+    for c in range(n):
+        got = set(np.nonzero(m[c])[0])
+        assert got == _brute_axis_window(n, w, c)
+        assert c in got and len(got) == min(w, n)
+        if w % 2 == 1 and c - w // 2 >= 0 and c + w // 2 <= n - 1:
+            assert got == {cc for cc in range(n) if abs(cc - c) <= w // 2}
+        if w % 2 == 1:   # reflection symmetry for centred (odd) windows
+            assert {n - 1 - cc for cc in got} == set(np.nonzero(m[n - 1 - c])[0])
+
+
+def test_window_is_product_and_counts():
+    d = _desc(T=7, Y=9, X=10, tT=1, tY=2, tX=3, wT=3, wY=3, wX=5)
+    g = oracle.geometry(d)
+    M = oracle.window_mask(d)
+    coords = [(a, b, c) for a in range(g.nT) for b in range(g.nY) for c in range(g.nX)]
+    for i, (a, b, c) in enumerate(coords):
+        for j, (a2, b2, c2) in enumerate(coords):
+            want = (a2 in _brute_axis_window(g.nT, 3, a) and b2 in _brute_axis_window(g.nY, 3, b)
+                    and c2 in _brute_axis_window(g.nX, 5, c))
+            assert M[i, j] == want
+        assert M[i].sum() == min(3, g.nT) * min(3, g.nY) * min(5, g.nX)
+
+
+# ---------------------------------------------------------------------------
+# Step 4: union and attention
+# ---------------------------------------------------------------------------
+
+def test_union_counts_and_text_rows():
+    w = si.get_workload("tiny_f32")
+    d = with_overrides(w, L_text=40, wT=1, wY=3, wX=1, topk=3)
+    g = oracle.geometry(d)
+    x = si.make_inputs(d)
+    r = oracle.ssta_forward(d, *(x[k].numpy() for k in ("q", "k", "v", "q_text", "k_text", "v_text")))
+    win = oracle.window_mask(d)
+    kept = r["kept"]
+    W = int(win[0].sum())
+    assert g.n_text == 2
+    assert np.all(kept[:, :, g.NT:, :])                      # text queries attend everything
+    assert np.all(kept[:, :, : g.NT, g.NT:])                 # every query attends text
+    assert np.all(kept[:, :, : g.NT, : g.NT] >= win)         # window kept
+    assert np.all(kept[:, :, : g.NT, : g.NT] >= r["sel"])    # selection kept
+    c = kept[:, :, : g.NT, : g.NT].sum(-1)
+    assert np.all(c >= max(g.k, W)) and np.all(c <= min(g.NT, g.k + W))
+    np.testing.assert_array_equal(r["kv_cnt"], kept.sum(-1))
+
+
+def _sdpa_raster(d, q, k, v, qt, kt, vt, allowed):
+    """torch SDPA (float64) on raster tokens [+ text] with a token-level boolean mask."""
+    B, H = q.shape[:2]
+    L = d.T * d.Y * d.X
+    cat = lambda a, b: np.concatenate([a.reshape(B, H, L, d.D)] + ([b] if b is not None else []), axis=2)
+    Q, K, V = (torch.from_numpy(cat(a, b)) for a, b in ((q, qt), (k, kt), (v, vt)))
+    m = torch.from_numpy(allowed)
+    O = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=m)
+    s = (Q @ K.transpose(-1, -2)) / math.sqrt(d.D)
+    lse = torch.logsumexp(s.masked_fill(~m, -math.inf), dim=-1)
+    return O.numpy(), lse.numpy()
+
+
+def _raster_tile_of(d):
+    g = oracle.geometry(d)
+    t, y, x = np.meshgrid(np.arange(d.T), np.arange(d.Y), np.arange(d.X), indexing="ij")
+    return (((t // d.tT) * g.nY + y // d.tY) * g.nX + x // d.tX).reshape(-1)
+
+
+def _token_mask_from_tile_mask(d, kept):
+    """[B,H,Lr,Lr] token mask in raster(+text) order from a tile-level kept mask."""
+    g = oracle.geometry(d)
+    member = _raster_tile_of(d)
+    if d.L_text:
+        member = np.concatenate([member, g.NT + np.arange(d.L_text) // g.N])
+    return kept[:, :, member][:, :, :, member]
+
+
+def _run_oracle(d, x):
+    arrs = [x[k].double().numpy() if x[k] is not None else None
+            for k in ("q", "k", "v", "q_text", "k_text", "v_text")]
+    return arrs, oracle.ssta_forward(d, *arrs)
+
+
+def _check_against_sdpa(d, arrs, r, kept_tiles):
+    O_ref, lse_ref = _sdpa_raster(d, *arrs, _token_mask_from_tile_mask(d, kept_tiles))
+    B, H = arrs[0].shape[:2]
+    L = d.T * d.Y * d.X
+    got = np.concatenate([r["O_raster"].reshape(B, H, L, d.D)]
+                         + ([r["O_text"]] if d.L_text else []), axis=2)
+    np.testing.assert_allclose(got, O_ref, rtol=0, atol=1e-12)
+    lse_raster, lse_text = oracle.tile_unorder(d, r["LSE"][..., None])
+    lse_got = np.concatenate([lse_raster.reshape(B, H, L)] + ([lse_text[..., 0]] if d.L_text else []),
+                             axis=2)
+    np.testing.assert_allclose(lse_got, lse_ref, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("L_text", [0, 37])
+def test_dense_equivalence_whole_window(L_text):
+    # window covering the whole grid -> dense attention over every valid token
+    w = si.get_workload("tiny_f32")
+    d = with_overrides(w, T=5, Y=7, X=6, wT=9, wY=9, wX=9, topk=0, L_text=L_text, D=16)
+    arrs, r = _run_oracle(d, si.make_inputs(d))
+    g = oracle.geometry(d)
+    assert r["kept"].all()
+    _check_against_sdpa(d, arrs, r, np.ones((d.B, d.H, g.NQ, g.NQ), dtype=bool))
+
+
+def test_dense_equivalence_topk_all():
+    w = si.get_workload("tiny_f32")
+    d = with_overrides(w, topk=1000, D=16)
+    arrs, r = _run_oracle(d, si.make_inputs(d))
+    g = oracle.geometry(d)
+    assert r["kept"].all()
+    _check_against_sdpa(d, arrs, r, np.ones((d.B, d.H, g.NQ, g.NQ), dtype=bool))
+
+
+def test_block_diagonal_special_case():
+    # window = own tile and top-k = 0 -> attention inside each tile only
+    w = si.get_workload("tiny_f32")
+    d = with_overrides(w, T=5, Y=7, X=6, topk=0, D=16)
+    arrs, r = _run_oracle(d, si.make_inputs(d))
+    g = oracle.geometry(d)
+    eye = np.broadcast_to(np.eye(g.NQ, dtype=bool), (d.B, d.H, g.NQ, g.NQ))
+    np.testing.assert_array_equal(r["kept"], eye)
+    member = _raster_tile_of(d)
+    allowed = np.broadcast_to(member[:, None] == member[None, :], (d.B, d.H) + (len(member),) * 2)
+    O_ref, _ = _sdpa_raster(d, *arrs, np.ascontiguousarray(allowed))
+    np.testing.assert_allclose(r["O_raster"].reshape(O_ref.shape), O_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("L_text", [0, 20])
+def test_general_kept_set_equals_masked_sdpa(L_text):
+    w = si.get_workload("tiny_f32")
+    d = with_overrides(w, T=6, Y=9, X=8, topk=3, wT=1, wY=3, wX=1, L_text=L_text, D=16, H=3)
+    arrs, r = _run_oracle(d, si.make_inputs(d, seed=7))
+    _check_against_sdpa(d, arrs, r, r["kept"])
+    # rows sum to one: sum_j exp(s_j - LSE) over the kept valid keys
+    g = oracle.geometry(d)
+    valid = oracle.valid_token_mask(d)
+    qp, kp = r["qp"], r["kp"]
+    for i in (0, g.NQ - 1):
+        rows = slice(i * g.N, min((i + 1) * g.N, g.Lq))
+        keys = np.concatenate([np.arange(j * g.N, min((j + 1) * g.N, g.Lq))
+                               for j in np.nonzero(r["kept"][0, 1, i])[0]])
+        keys = keys[valid[keys]]
+        s = qp[0, 1, rows] @ kp[0, 1, keys].T / math.sqrt(d.D)
+        np.testing.assert_allclose(np.exp(s - r["LSE"][0, 1, rows, None]).sum(1), 1.0, atol=1e-12)
+
+
+def test_whole_mask_brute_force_tiny():
+    # pooled means, scores, top-k, window and union rebuilt from raster data by brute force
+    d = si.get_workload("tiny_f32")
+    x = si.make_inputs(d)
+    arrs, r = _run_oracle(d, x)
+    g = oracle.geometry(d)
+    member = _raster_tile_of(d)
+    for h in range(d.H):
+        qf = arrs[0][0, h].reshape(-1, d.D)
+        kf = arrs[1][0, h].reshape(-1, d.D)
+        qb = np.stack([qf[member == c].mean(0) for c in range(g.NT)])
+        kb = np.stack([kf[member == c].mean(0) for c in range(g.NT)])
+        S = qb @ kb.T
+        for i in range(g.NT):
+            sel = _brute_topk(S[i].astype(np.float32), g.k)
+            a, b, c = i // (g.nY * g.nX), (i // g.nX) % g.nY, i % g.nX
+            win = {(a2 * g.nY + b2) * g.nX + c2
+                   for a2 in _brute_axis_window(g.nT, d.wT, a)
+                   for b2 in _brute_axis_window(g.nY, d.wY, b)
+                   for c2 in _brute_axis_window(g.nX, d.wX, c)}
+            assert set(np.nonzero(r["kept"][0, h, i])[0]) == sel | win
+
+
+def test_flop_count_dense_case():
+    w = si.get_workload("tiny_f32")
+    g = oracle.geometry(w)
+    kept = np.ones((1, w.H, g.NQ, g.NQ), dtype=bool)
+    L = w.T * w.Y * w.X
+    assert oracle.attention_flops(w, kept) == 4.0 * w.D * w.H * L * L

@@ -1,0 +1,73 @@
+// Internal declarations shared by the SSTA CUDA translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ssta.h"
+
+namespace ssta {
+
+// Every size the kernels need, derived once on the host from an ssta_desc.
+struct Geom {
+  int B, H, D;
+  int T, Y, X;          // valid grid
+  int tT, tY, tX;       // tile extents
+  int nT, nY, nX;       // tiles per axis
+  int N;                // tokens per tile
+  int NT;               // video tiles
+  int L_text;
+  int n_text;           // text tiles
+  int NQ;               // query tiles
+  int64_t Lq;           // packed length
+  int k;                // top-k, clamped
+  int wT, wY, wX;       // window (tiles)
+  int window_tiles;
+  int max_kept;
+  int words;            // 32-bit words per selection-bitset row = ceil(NT/32)
+  int esize;            // bytes per element (2 or 4)
+  int dtype;
+  float scale;          // softmax scale
+};
+
+// Workspace layout of ssta_build_block_mask (byte offsets, 256-aligned).
+struct MaskWorkspace {
+  size_t status;   // int32 device status word
+  size_t qbar;     // fp32 [BH, NT, D]
+  size_t kbar;     // fp32 [BH, NT, D]
+  size_t scores;   // fp32 [BH, NT, NT]
+  size_t selbits;  // u32  [BH, NT, words]
+  size_t total;
+};
+
+MaskWorkspace mask_workspace_layout(const Geom& g);
+
+// Launchers (return cudaGetLastError() of their launches).
+cudaError_t launch_tile_reorder(const Geom& g, const void* raster, const void* text, void* packed,
+                                cudaStream_t s);
+cudaError_t launch_tile_unorder(const Geom& g, const void* packed, void* raster, void* text,
+                                cudaStream_t s);
+cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, float* qbar, float* kbar,
+                             cudaStream_t s);
+cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
+                               cudaStream_t s);
+cudaError_t launch_select_topk(const Geom& g, const float* scores, uint32_t* selbits, cudaStream_t s);
+cudaError_t launch_build_kv_lists(const Geom& g, const uint32_t* selbits, int32_t* kv_idx,
+                                  int32_t* kv_cnt, cudaStream_t s);
+cudaError_t launch_attention_f32(const Geom& g, const float* qp, const float* kp, const float* vp,
+                                 const int32_t* kv_idx, const int32_t* kv_cnt, float* o, float* lse,
+                                 int32_t* status, cudaStream_t s);
+cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* kp, const void* vp,
+                                     const int32_t* kv_idx, const int32_t* kv_cnt, void* o, float* lse,
+                                     int32_t* status, cudaStream_t s);
+
+// Device-side helpers shared by kernels.
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Number of valid tokens along one axis of tile coordinate c (tile extent t, valid extent n).
+__host__ __device__ inline int axis_valid(int c, int t, int n) {
+  int v = n - c * t;
+  return v < t ? v : t;
+}
+
+}  // namespace ssta

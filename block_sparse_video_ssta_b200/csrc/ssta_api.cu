@@ -14,6 +14,10 @@ constexpr int kMaxTiles = 2048;        // NT; one warp holds a score row in regi
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+ssta_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH; }
+
+}  // namespace
+
 // Host-side geometry (Step 1, "3D Block Partition").  Returns SSTA_OK or the
 // reason the descriptor is rejected.
 ssta_status make_geom(const ssta_desc* d, Geom* g) {
@@ -62,9 +66,6 @@ ssta_status make_geom(const ssta_desc* d, Geom* g) {
   return SSTA_OK;
 }
 
-ssta_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH; }
-
-}  // namespace
 }  // namespace ssta
 
 using namespace ssta;

@@ -42,6 +42,9 @@ struct MaskWorkspace {
 
 MaskWorkspace mask_workspace_layout(const Geom& g);
 
+// Validate a descriptor and derive every size (host only, no CUDA call).
+ssta_status make_geom(const ssta_desc* d, Geom* g);
+
 // Launchers (return cudaGetLastError() of their launches).
 cudaError_t launch_tile_reorder(const Geom& g, const void* raster, const void* text, void* packed,
                                 cudaStream_t s);

@@ -158,6 +158,26 @@ ssta_status ssta_tile_unorder(const ssta_desc* desc, const void* x_packed, void*
                               void* x_text, void* stream);
 
 /*
+ * ssta_build_block_mask_noalloc — the same computation and outputs as
+ * ssta_build_block_mask, for callers that cannot allocate device memory at call
+ * time (for instance a plugin that an inference engine hands only pre-planned
+ * tensors, or a service that reserved all device memory for its own pool).  The
+ * paper has no counterpart to this call; it exists for those callers only.
+ *   Scratch: a device array of SSTA_STATIC_SCRATCH_BYTES built into the library,
+ *   one per GPU that loads it, resident until the process exits.  Problems whose
+ *   scratch would exceed it (status word, pooled q and k, the score matrix
+ *   unless tile_scores is given, selection bits) return SSTA_ERR_WORKSPACE.
+ *   The call allocates nothing.  All calls on a device share the array, so calls
+ *   whose kernels overlap on the GPU race: serialise them.  The first call on a
+ *   device looks up the array's device address (with that device current); make
+ *   it before any stream capture.
+ *   Arguments as for ssta_build_block_mask, without the workspace.
+ */
+#define SSTA_STATIC_SCRATCH_BYTES (32u << 20)
+ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, const void* q_packed, const void* k_packed,
+                                          int32_t* kv_idx, int32_t* kv_cnt, float* tile_scores, void* stream);
+
+/*
  * ssta_read_device_status — copy the device status word (first int32 of a
  * workspace used by the calls above) to *code, synchronising `stream` first.
  * Diagnostic call: the only function of this library that synchronises.

@@ -18,8 +18,10 @@
 //   O_h = sum P V  fp32, columns [256+128h, 256+128h+128)
 // MMA schedule per chunk j (the next chunk's S overlaps the softmax of the
 // other half):  PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).
-// Softmax: base-2 exponentials with the scale folded in, running max and sum
-// in fp32; O is rescaled in TMEM only when a warp's running max moved.
+// Softmax: one 128-column TMEM load per chunk, base-2 exponentials with the
+// scale folded in, running max and sum in fp32; the reference max moves only
+// when the row max exceeds it by more than 8 (probabilities stay below 2^8),
+// so O is rescaled in TMEM rarely.
 //
 // Every mbarrier wait is bounded in time.  A wait that runs out records
 // SSTA_ERR_DEVICE_TIMEOUT in the status word, raises a CTA-wide abort flag that
@@ -163,16 +165,31 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&p)[16]) {
+// 128 consecutive TMEM columns of this thread's lane in one load, waited in the same asm block.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+  uint32_t r[128];
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
-      ::"r"(taddr), "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7]),
-        "r"(p[8]), "r"(p[9]), "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15])
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&p)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};"
+      ::"r"(taddr), "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7]), "r"(p[8]), "r"(p[9]), "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15]), "r"(p[16]), "r"(p[17]), "r"(p[18]), "r"(p[19]), "r"(p[20]), "r"(p[21]), "r"(p[22]), "r"(p[23]), "r"(p[24]), "r"(p[25]), "r"(p[26]), "r"(p[27]), "r"(p[28]), "r"(p[29]), "r"(p[30]), "r"(p[31]), "r"(p[32]), "r"(p[33]), "r"(p[34]), "r"(p[35]), "r"(p[36]), "r"(p[37]), "r"(p[38]), "r"(p[39]), "r"(p[40]), "r"(p[41]), "r"(p[42]), "r"(p[43]), "r"(p[44]), "r"(p[45]), "r"(p[46]), "r"(p[47]), "r"(p[48]), "r"(p[49]), "r"(p[50]), "r"(p[51]), "r"(p[52]), "r"(p[53]), "r"(p[54]), "r"(p[55]), "r"(p[56]), "r"(p[57]), "r"(p[58]), "r"(p[59]), "r"(p[60]), "r"(p[61]), "r"(p[62]), "r"(p[63])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -480,43 +497,54 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
     const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool full) -> bool {
       if (!wait_warp(bar(BAR_SFULL + h), (uint32_t)(j & 1), ctl)) return false;
       tc_fence_after();
-      uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
+      float sv[128];
+      tmem_ld128(tSh, sv);
       if (!full) {
+        // pad keys of this chunk (same columns for every row) never enter the softmax
 #pragma unroll
-        for (int q = 0; q < 4; ++q) vm[q] = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + q * 32 + lane));
-      }
-      float v[32];
-      float mx = -INFINITY;
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t vm = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + q * 32 + lane));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        tmem_ld32(tSh + 32u * q, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((vm[q] >> i) & 1u) mx = fmaxf(mx, v[i]);
-      }
-      const float m_new = fmaxf(m, mx * scale_log2);
-      const float alpha = ex2(m - m_new);
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        tmem_ld32(tSh + 32u * q, v);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ((vm[q] >> (2 * i)) & 1u) ? ex2(fmaf(v[2 * i], scale_log2, -m_new)) : 0.f;
-          const float p1 = ((vm[q] >> (2 * i + 1)) & 1u) ? ex2(fmaf(v[2 * i + 1], scale_log2, -m_new)) : 0.f;
-          sum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 32; ++i)
+            if (!((vm >> i) & 1u)) sv[q * 32 + i] = -INFINITY;
         }
-        tmem_st16(tSh + 16u * q, pk);
       }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(sv[i], sv[i + 8]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], sv[i + k], sv[i + 8 + k]);
+      const float rmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+                         scale_log2;
+      // Lazy rescaling: the reference max only moves when the row max exceeds it by more
+      // than 8 (base 2), so probabilities stay below 2^8 and O is rescaled rarely.
+      const bool moved = rmax > m + 8.0f;
+      const float m_new = moved ? rmax : m;
+      const float alpha = moved ? ex2(m - m_new) : 1.0f;
+      m = m_new;
+      const float neg_m = -m_new;
+      float sum[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum[i] = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2(fmaf(sv[2 * i], scale_log2, neg_m));
+        const float p1 = ex2(fmaf(sv[2 * i + 1], scale_log2, neg_m));
+        sum[i & 7] += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      tmem_st64(tSh, pk);
       tmem_wait_st();
-      l = l * alpha + sum;
-      if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
+      l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
+      if (j > 0 && __any_sync(0xffffffffu, moved)) {
         if (!wait_warp(bar(BAR_ODONE + h), (uint32_t)((j - 1) & 1), ctl)) return false;
         tc_fence_after();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          float v[32];
           tmem_ld32(tOh + 32u * q, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= alpha;
@@ -524,7 +552,6 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         }
         tmem_wait_st();
       }
-      m = m_new;
       tc_fence_before();
       mbar_arrive(bar(BAR_PREADY + h));
       return true;

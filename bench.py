@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "SSTA fwd ms/call & effective TFLOPS (kept blocks) at 720p-10s latent; % bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-LAUNCHES_PER_STEP = 9   # 3 reorder + pool + scores + top-k + lists + attention + unorder
+LAUNCHES_PER_STEP = 8   # 3 reorder + pool + scores + select-and-list + attention + unorder
 
 
 def load_peaks():

@@ -136,11 +136,9 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
   float* qbar = reinterpret_cast<float*>(w + ws.qbar);
   float* kbar = reinterpret_cast<float*>(w + ws.kbar);
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(w + ws.scores);
-  uint32_t* sel = reinterpret_cast<uint32_t*>(w + ws.selbits);
   cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, scores, s);
-  if (e == cudaSuccess) e = launch_select_topk(g, scores, sel, s);
-  if (e == cudaSuccess) e = launch_build_kv_lists(g, sel, kv_idx, kv_cnt, s);
+  if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return from_cuda(e);
 }
 

@@ -19,9 +19,10 @@
 // MMA schedule per chunk j (the next chunk's S overlaps the softmax of the
 // other half):  PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).
 // Softmax: one 128-column TMEM load per chunk, base-2 exponentials with the
-// scale folded in, running max and sum in fp32; the reference max moves only
-// when the row max exceeds it by more than 8 (probabilities stay below 2^8),
-// so O is rescaled in TMEM rarely.
+// scale folded in, running max and sum in fp32 (scale-and-shift and the row sum
+// two lanes per instruction with f32x2); the reference max moves only when the
+// row max exceeds it by more than 8 (probabilities stay below 2^8), so O is
+// rescaled in TMEM rarely.
 //
 // Every mbarrier wait is bounded in time.  A wait that runs out records
 // SSTA_ERR_DEVICE_TIMEOUT in the status word, raises a CTA-wide abort flag that
@@ -194,6 +195,25 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// Two-lane fp32 arithmetic (sm_100): one instruction for a pair of values.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -525,17 +545,23 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
       const float alpha = moved ? ex2(m - m_new) : 1.0f;
       m = m_new;
       const float neg_m = -m_new;
-      float sum[8];
+      // scale-and-shift and the row sum run two lanes per instruction (f32x2)
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(neg_m, neg_m);
+      uint64_t sum2[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum[i] = 0.f;
+      for (int i = 0; i < 4; ++i) sum2[i] = f2_pack(0.f, 0.f);
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(fmaf(sv[2 * i], scale_log2, neg_m));
-        const float p1 = ex2(fmaf(sv[2 * i + 1], scale_log2, neg_m));
-        sum[i & 7] += p0 + p1;
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), c2, nm2), x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(p0, p1));
         pk[i] = pack_bf16x2(p0, p1);
       }
+      float sum[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f2_unpack(sum2[i], sum[2 * i], sum[2 * i + 1]);
       tmem_st64(tSh, pk);
       tmem_wait_st();
       l = l * alpha + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));

@@ -33,10 +33,9 @@ struct Geom {
 // Workspace layout of ssta_build_block_mask (byte offsets, 256-aligned).
 struct MaskWorkspace {
   size_t status;   // int32 device status word
-  size_t qbar;     // fp32 [BH, NT, D]
-  size_t kbar;     // fp32 [BH, NT, D]
+  size_t qbar;     // fp32 [BH, D, NT] (channel-major)
+  size_t kbar;     // fp32 [BH, D, NT] (channel-major)
   size_t scores;   // fp32 [BH, NT, NT]
-  size_t selbits;  // u32  [BH, NT, words]
   size_t total;
 };
 
@@ -54,9 +53,8 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
                              cudaStream_t s);
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
                                cudaStream_t s);
-cudaError_t launch_select_topk(const Geom& g, const float* scores, uint32_t* selbits, cudaStream_t s);
-cudaError_t launch_build_kv_lists(const Geom& g, const uint32_t* selbits, int32_t* kv_idx,
-                                  int32_t* kv_cnt, cudaStream_t s);
+cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
+                                   cudaStream_t s);
 cudaError_t launch_attention_f32(const Geom& g, const float* qp, const float* kp, const float* vp,
                                  const int32_t* kv_idx, const int32_t* kv_cnt, float* o, float* lse,
                                  int32_t* status, cudaStream_t s);

@@ -9,18 +9,18 @@
 // Kernels, in launch order:
 //   tile_pool_kernel      HBM-bound: one CTA per (head, tile) streams the tile's
 //                         valid q and k rows with 16-byte coalesced loads and
-//                         reduces per-channel fp32 sums across row groups.
-//   tile_scores_kernel    fp32 SIMT, 64x64 score blocks per CTA, channels
-//                         summed in order 0..D-1 with FMA.
-//   select_topk_kernel    one warp per (head, query tile): scores held in
-//                         registers as order-preserving 32-bit keys, k-th key
-//                         found by a bitwise binary search with warp-wide
-//                         counts, ties resolved to the lower tile index by
-//                         ballots in index order; writes a selection bitset.
-//   build_kv_lists_kernel one warp per (head, query tile): window membership
-//                         computed per candidate, OR-ed with the bitset and the
-//                         text tiles, compacted in ascending order by ballot
-//                         prefix counts.
+//                         reduces per-channel fp32 sums across row groups; the
+//                         means are stored channel-major for the score kernel.
+//   tile_scores_kernel    fp32 SIMT, 128x64 score blocks per CTA, 32 channels at
+//                         a time in shared memory, channels summed in order
+//                         0..D-1 with FMA.
+//   select_and_list_kernel one warp per (head, query tile): top-k over scores
+//                         held in registers as order-preserving 32-bit keys
+//                         (bitwise binary search for the k-th key with warp-wide
+//                         counts, ties to the lower tile index by ballots in
+//                         index order), OR-ed word by word with the window
+//                         (contiguous index ranges) and compacted into the
+//                         ascending kept list by a warp prefix sum.
 #include "ssta_internal.h"
 
 #include <cuda_bf16.h>
@@ -113,60 +113,72 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
     float s = 0.f;
     for (int r = 0; r < rpp; ++r) s += red[(which * rpp + r) * D + ch];
     float* out = which ? kbar : qbar;
-    out[(bh * g.NT + c) * D + ch] = s * inv;
+    out[(bh * D + ch) * g.NT + c] = s * inv;     // channel-major: [head][channel][tile]
   }
 }
 
-// Step 2, Score_s = Qbar Kbar^T: 64x64 output block per CTA, 16x16 threads,
-// each thread 4x4 outputs at stride 16; channels in chunks of 32 via smem.
-constexpr int kScoreTile = 64;
+// Step 2, Score_s = Qbar Kbar^T.  One CTA computes a 128 x 64 block of scores for
+// one head; 256 threads as 16 x 16, each owning 8 rows x 4 columns.  The pooled
+// means arrive channel-major ([head][channel][tile]), so 32 channels at a time are
+// copied into shared memory with coalesced loads in the same layout, and a thread's
+// 8 + 4 operands for one channel are three 16-byte loads feeding 32 FMAs.  Every
+// score is accumulated over channels 0..D-1 in order with FMA.
+constexpr int kScoreRows = 128;
+constexpr int kScoreCols = 64;
 constexpr int kScoreChunk = 32;
 
 __global__ void __launch_bounds__(256)
-tile_scores_kernel(Geom g, const float* __restrict__ qbar, const float* __restrict__ kbar,
+tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __restrict__ kbar_t,
                    float* __restrict__ scores) {
-  __shared__ float qs[kScoreTile][kScoreChunk + 1];
-  __shared__ float ks[kScoreTile][kScoreChunk + 1];
+  __shared__ __align__(16) float qs[kScoreChunk][kScoreRows + 4];
+  __shared__ __align__(16) float ks[kScoreChunk][kScoreCols + 4];
   const int64_t bh = blockIdx.z;
-  const int i0 = blockIdx.y * kScoreTile, j0 = blockIdx.x * kScoreTile;
+  const int i0 = blockIdx.y * kScoreRows, j0 = blockIdx.x * kScoreCols;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const float* qh = qbar + bh * g.NT * g.D;
-  const float* kh = kbar + bh * g.NT * g.D;
-  float acc[4][4];
+  const float* qh = qbar_t + bh * g.D * (int64_t)g.NT;
+  const float* kh = kbar_t + bh * g.D * (int64_t)g.NT;
+  float acc[8][4];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
 
   for (int d0 = 0; d0 < g.D; d0 += kScoreChunk) {
-    for (int e = threadIdx.x; e < kScoreTile * kScoreChunk; e += 256) {
-      const int r = e / kScoreChunk, cc = e % kScoreChunk;
-      qs[r][cc] = (i0 + r < g.NT) ? qh[(int64_t)(i0 + r) * g.D + d0 + cc] : 0.f;
-      ks[r][cc] = (j0 + r < g.NT) ? kh[(int64_t)(j0 + r) * g.D + d0 + cc] : 0.f;
+    for (int e = threadIdx.x; e < kScoreChunk * kScoreRows; e += 256) {
+      const int cc = e / kScoreRows, r = e % kScoreRows, i = i0 + r;
+      qs[cc][r] = i < g.NT ? __ldg(qh + (int64_t)(d0 + cc) * g.NT + i) : 0.f;
+    }
+    for (int e = threadIdx.x; e < kScoreChunk * kScoreCols; e += 256) {
+      const int cc = e / kScoreCols, r = e % kScoreCols, j = j0 + r;
+      ks[cc][r] = j < g.NT ? __ldg(kh + (int64_t)(d0 + cc) * g.NT + j) : 0.f;
     }
     __syncthreads();
-#pragma unroll 8
+#pragma unroll 4
     for (int cc = 0; cc < kScoreChunk; ++cc) {
-      float qv[4], kv[4];
+      const float4 qa = *reinterpret_cast<const float4*>(&qs[cc][ty * 8]);
+      const float4 qb = *reinterpret_cast<const float4*>(&qs[cc][ty * 8 + 4]);
+      const float4 kv = *reinterpret_cast<const float4*>(&ks[cc][tx * 4]);
+      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+      const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qv[a] = qs[ty + 16 * a][cc];
+      for (int a = 0; a < 8; ++a)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kv[b] = ks[tx + 16 * b][cc];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], kk[b], acc[a][b]);
     }
     __syncthreads();
   }
   float* sh = scores + bh * g.NT * (int64_t)g.NT;
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty + 16 * a;
+  for (int a = 0; a < 8; ++a) {
+    const int i = i0 + ty * 8 + a;
+    if (i >= g.NT) continue;
+    const int j = j0 + tx * 4;
+    if (j + 3 < g.NT && (g.NT % 4) == 0) {
+      *reinterpret_cast<float4*>(sh + (int64_t)i * g.NT + j) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    } else {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = j0 + tx + 16 * b;
-      if (i < g.NT && j < g.NT) sh[(int64_t)i * g.NT + j] = acc[a][b];
+      for (int b = 0; b < 4; ++b)
+        if (j + b < g.NT) sh[(int64_t)i * g.NT + j + b] = acc[a][b];
     }
   }
 }
@@ -178,57 +190,6 @@ __device__ __forceinline__ uint32_t float_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Step 2, Topk + Indexes2mask.  One warp per (head, query tile); candidate j
-// sits in lane j % 32, slot j / 32.
-template <int SLOTS>
-__global__ void __launch_bounds__(256)
-select_topk_kernel(Geom g, const float* __restrict__ scores, uint32_t* __restrict__ selbits) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // bh * NT + i
-  if (row >= (int64_t)g.B * g.H * g.NT) return;
-  const float* s = scores + row * g.NT;
-  uint32_t* out = selbits + row * g.words;
-  const int k = g.k;
-  uint32_t key[SLOTS];
-#pragma unroll
-  for (int w = 0; w < SLOTS; ++w) {
-    const int j = w * 32 + lane;
-    key[w] = (w < g.words && j < g.NT) ? float_key(s[j]) : 0u;   // 0 is below every real key
-  }
-  if (k == 0) {
-    for (int w = lane; w < g.words; w += 32) out[w] = 0u;
-    return;
-  }
-  // Largest threshold thr with #(key >= thr) >= k: the k-th largest key.
-  uint32_t thr = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = thr | (1u << bit);
-    int cnt = 0;
-#pragma unroll
-    for (int w = 0; w < SLOTS; ++w) cnt += (key[w] >= cand) ? 1 : 0;
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (cnt >= k) thr = cand;
-  }
-  int gt = 0;
-#pragma unroll
-  for (int w = 0; w < SLOTS; ++w) gt += (key[w] > thr) ? 1 : 0;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const int need = k - gt;          // equal keys to take, lowest tile index first
-  int eq_before = 0;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-#pragma unroll
-  for (int w = 0; w < SLOTS; ++w) {
-    if (w < g.words) {
-      const bool eq = key[w] == thr;
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-      const bool take = key[w] > thr || (eq && eq_before + __popc(eqm & lt_mask) < need);
-      const uint32_t word = __ballot_sync(0xffffffffu, take);
-      if (lane == 0) out[w] = word;
-      eq_before += __popc(eqm);
-    }
-  }
-}
-
 // Per-axis window start: the window of span min(w, n) slides inward at the edges.
 __device__ __forceinline__ int window_start(int c, int w, int n) {
   const int span = w < n ? w : n;
@@ -237,10 +198,33 @@ __device__ __forceinline__ int window_start(int c, int w, int n) {
   return s > n - span ? n - span : s;
 }
 
-// Steps 3-4: union of selection, window and text tiles -> ascending lists.
+// Bits of tile indices [32*word, 32*word+32) that fall in [lo, hi).
+__device__ __forceinline__ uint32_t range_bits(int word, int lo, int hi) {
+  const int a = max(lo - 32 * word, 0), b = min(hi - 32 * word, 32);
+  if (a >= b) return 0u;
+  const uint32_t upto_b = b == 32 ? 0xffffffffu : ((1u << b) - 1u);
+  return upto_b & ~((1u << a) - 1u);
+}
+
+// Steps 2-4 for one (head, query tile) per warp:
+//  * Topk + Indexes2mask (video query tiles): the scores of the row are held in
+//    registers as order-preserving 32-bit keys (candidate j in lane j % 32, slot
+//    j / 32); the k-th largest key is found by a bitwise binary search with
+//    warp-wide counts (upper 16 bits over all keys, lower 16 bits over the keys
+//    sharing that upper half); keys above it are taken, and keys equal to it are
+//    taken in ascending tile order until k are chosen (ties to the lower index);
+//  * the window (Step 3) as unions of contiguous index ranges, one per (t, y)
+//    tile row of the window, OR-ed word by word with the selection;
+//  * the union (Step 4) written as an ascending list by a warp prefix sum over the
+//    32-tile words, followed by the text tiles and -1 padding.
+// Text query tiles keep every tile.
+constexpr int kBucketCap = 64;
+
+template <int SLOTS>
 __global__ void __launch_bounds__(256)
-build_kv_lists_kernel(Geom g, const uint32_t* __restrict__ selbits, int32_t* __restrict__ kv_idx,
-                      int32_t* __restrict__ kv_cnt) {
+select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __restrict__ kv_idx,
+                       int32_t* __restrict__ kv_cnt) {
+  __shared__ uint32_t bucket_smem[8 * kBucketCap];
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // bh * NQ + i
   if (row >= (int64_t)g.B * g.H * g.NQ) return;
@@ -250,22 +234,121 @@ build_kv_lists_kernel(Geom g, const uint32_t* __restrict__ selbits, int32_t* __r
   const uint32_t lt_mask = (1u << lane) - 1u;
   int base = 0;
   if (i < g.NT) {
+    // ---- selection
+    const float* srow = scores + (bh * g.NT + i) * (int64_t)g.NT;
+    uint32_t key[SLOTS];
+#pragma unroll
+    for (int w = 0; w < SLOTS; ++w) {
+      const int j = w * 32 + lane;
+      key[w] = (w < g.words && j < g.NT) ? float_key(srow[j]) : 0u;   // 0 is below every real key
+    }
+    uint32_t myword[(SLOTS + 31) / 32];   // lane holds selection words lane and lane + 32
+#pragma unroll
+    for (int q = 0; q < (SLOTS + 31) / 32; ++q) myword[q] = 0u;
+    const int k = g.k;
+    if (k > 0) {
+      // k-th largest key in two levels: a bitwise search over the upper 16 bits of every
+      // key, then over the lower 16 bits of the keys that share the found upper half
+      // (the boundary bucket, compacted into shared memory when it holds at most 64;
+      // otherwise the lower bits are searched over all keys).
+      uint32_t hi = 0;
+      for (int bit = 15; bit >= 0; --bit) {
+        const uint32_t cand = (hi | (1u << bit)) << 16;
+        int cnt = 0;
+#pragma unroll
+        for (int w = 0; w < SLOTS; ++w) cnt += (key[w] >= cand) ? 1 : 0;
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (cnt >= k) hi |= 1u << bit;
+      }
+      int above = 0, bsize = 0;
+      uint32_t* bucket = bucket_smem + (threadIdx.x >> 5) * kBucketCap;
+#pragma unroll
+      for (int w = 0; w < SLOTS; ++w) {
+        above += ((key[w] >> 16) > hi) ? 1 : 0;
+        const bool in = key[w] != 0u && (key[w] >> 16) == hi;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        const int pos = bsize + __popc(m & lt_mask);
+        if (in && pos < kBucketCap) bucket[pos] = key[w];
+        bsize += __popc(m);
+      }
+      above = __reduce_add_sync(0xffffffffu, above);
+      __syncwarp();
+      const int need_lo = k - above;     // keys to take from the bucket (>= 1)
+      uint32_t thr = hi << 16;
+      if (bsize <= kBucketCap) {
+        const uint32_t b0 = lane < bsize ? bucket[lane] : 0u;
+        const uint32_t b1 = lane + 32 < bsize ? bucket[lane + 32] : 0u;
+        for (int bit = 15; bit >= 0; --bit) {
+          const uint32_t cand = thr | (1u << bit);
+          const int cnt = __reduce_add_sync(0xffffffffu, (b0 >= cand ? 1 : 0) + (b1 >= cand ? 1 : 0));
+          if (cnt >= need_lo) thr = cand;
+        }
+      } else {
+        for (int bit = 15; bit >= 0; --bit) {
+          const uint32_t cand = thr | (1u << bit);
+          int cnt = 0;
+#pragma unroll
+          for (int w = 0; w < SLOTS; ++w) cnt += (key[w] >= cand) ? 1 : 0;
+          cnt = __reduce_add_sync(0xffffffffu, cnt);
+          if (cnt >= k) thr = cand;
+        }
+      }
+      __syncwarp();
+      int gt = 0;
+#pragma unroll
+      for (int w = 0; w < SLOTS; ++w) gt += (key[w] > thr) ? 1 : 0;
+      gt = __reduce_add_sync(0xffffffffu, gt);
+      const int need = k - gt;
+      int eq_before = 0;
+#pragma unroll
+      for (int w = 0; w < SLOTS; ++w) {
+        if (w < g.words) {
+          const bool eq = key[w] == thr;
+          const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+          const bool take = key[w] > thr || (eq && eq_before + __popc(eqm & lt_mask) < need);
+          const uint32_t word = __ballot_sync(0xffffffffu, take);
+          if ((w & 31) == lane) myword[w >> 5] = word;
+          eq_before += __popc(eqm);
+        }
+      }
+    }
+    // ---- window rows: for each (t, y) tile row of the window, a contiguous x range
     const int cX = i % g.nX, cY = (i / g.nX) % g.nY, cT = i / (g.nX * g.nY);
     const int sT = window_start(cT, g.wT, g.nT), sY = window_start(cY, g.wY, g.nY),
               sX = window_start(cX, g.wX, g.nX);
-    const int eT = sT + min(g.wT, g.nT), eY = sY + min(g.wY, g.nY), eX = sX + min(g.wX, g.nX);
-    const uint32_t* bits = selbits + (bh * g.NT + i) * g.words;
-    for (int w = 0; w < g.words; ++w) {
-      const int j = w * 32 + lane;
-      bool keep = false;
-      if (j < g.NT) {
-        const int jX = j % g.nX, jY = (j / g.nX) % g.nY, jT = j / (g.nX * g.nY);
-        const bool in_win = jT >= sT && jT < eT && jY >= sY && jY < eY && jX >= sX && jX < eX;
-        keep = in_win || ((bits[w] >> lane) & 1u);
+    const int eT = sT + min(g.wT, g.nT), eY = sY + min(g.wY, g.nY), nwX = min(g.wX, g.nX);
+#pragma unroll
+    for (int q = 0; q < (SLOTS + 31) / 32; ++q) {
+      const int word = lane + 32 * q;
+      if (word >= g.words) continue;
+      uint32_t win = 0u;
+      for (int wt = sT; wt < eT; ++wt)
+        for (int wy = sY; wy < eY; ++wy) {
+          const int lo = (wt * g.nY + wy) * g.nX + sX;
+          win |= range_bits(word, lo, lo + nwX);
+        }
+      myword[q] |= win;
+    }
+    // ---- compaction: exclusive prefix of the kept counts over words in ascending order
+#pragma unroll
+    for (int q = 0; q < (SLOTS + 31) / 32; ++q) {
+      const int word = lane + 32 * q;
+      const uint32_t bits = word < g.words ? myword[q] : 0u;
+      int c = __popc(bits);
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
       }
-      const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      if (keep) out[base + __popc(m & lt_mask)] = j;
-      base += __popc(m);
+      int pos = base + incl - c;
+      uint32_t rest = bits;
+      while (rest) {
+        const int b = __ffs(rest) - 1;
+        rest &= rest - 1u;
+        out[pos++] = 32 * word + b;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
     }
     for (int t = lane; t < g.n_text; t += 32) out[base + t] = g.NT + t;
     base += g.n_text;
@@ -289,8 +372,7 @@ MaskWorkspace mask_workspace_layout(const Geom& g) {
   w.qbar = 256;
   w.kbar = w.qbar + up(bh * g.NT * g.D * sizeof(float));
   w.scores = w.kbar + up(bh * g.NT * g.D * sizeof(float));
-  w.selbits = w.scores + up(bh * g.NT * (size_t)g.NT * sizeof(float));
-  w.total = w.selbits + up(bh * g.NT * (size_t)g.words * sizeof(uint32_t));
+  w.total = w.scores + up(bh * g.NT * (size_t)g.NT * sizeof(float));
   return w;
 }
 
@@ -313,31 +395,24 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
                                cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
-  dim3 grid(ceil_div(g.NT, kScoreTile), ceil_div(g.NT, kScoreTile), g.B * g.H);
+  dim3 grid(ceil_div(g.NT, kScoreCols), ceil_div(g.NT, kScoreRows), g.B * g.H);
   tile_scores_kernel<<<grid, 256, 0, s>>>(g, qbar, kbar, scores);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select_topk(const Geom& g, const float* scores, uint32_t* selbits, cudaStream_t s) {
-  const int64_t rows = (int64_t)g.B * g.H * g.NT;
+cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
+                                   cudaStream_t s) {
+  const int64_t rows = (int64_t)g.B * g.H * g.NQ;
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((rows + 7) / 8);
   if (g.words <= 8)
-    select_topk_kernel<8><<<blocks, 256, 0, s>>>(g, scores, selbits);
+    select_and_list_kernel<8><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
   else if (g.words <= 16)
-    select_topk_kernel<16><<<blocks, 256, 0, s>>>(g, scores, selbits);
+    select_and_list_kernel<16><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
   else if (g.words <= 32)
-    select_topk_kernel<32><<<blocks, 256, 0, s>>>(g, scores, selbits);
+    select_and_list_kernel<32><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
   else
-    select_topk_kernel<64><<<blocks, 256, 0, s>>>(g, scores, selbits);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_build_kv_lists(const Geom& g, const uint32_t* selbits, int32_t* kv_idx,
-                                  int32_t* kv_cnt, cudaStream_t s) {
-  const int64_t rows = (int64_t)g.B * g.H * g.NQ;
-  if (rows == 0) return cudaSuccess;
-  build_kv_lists_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(g, selbits, kv_idx, kv_cnt);
+    select_and_list_kernel<64><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 

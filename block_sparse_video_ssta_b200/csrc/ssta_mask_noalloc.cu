@@ -62,14 +62,13 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
-  // scratch layout: status word | qbar | kbar | scores (only without tile_scores) | selection bits
+  // scratch layout: status word | qbar | kbar | scores (only without tile_scores)
   const size_t bh = (size_t)g.B * g.H;
   const size_t off_qbar = 256;
   const size_t off_kbar = off_qbar + up256(bh * g.NT * g.D * sizeof(float));
   const size_t off_scores = off_kbar + up256(bh * g.NT * g.D * sizeof(float));
   const size_t scores_bytes = tile_scores != nullptr ? 0 : up256(bh * g.NT * (size_t)g.NT * sizeof(float));
-  const size_t off_sel = off_scores + scores_bytes;
-  const size_t total = off_sel + up256(bh * g.NT * (size_t)g.words * sizeof(uint32_t));
+  const size_t total = off_scores + scores_bytes;
   if (total > (size_t)SSTA_STATIC_SCRATCH_BYTES) return SSTA_ERR_WORKSPACE;
   const bool empty = bh == 0;
   if (!empty && (q_packed == nullptr || k_packed == nullptr || kv_idx == nullptr || kv_cnt == nullptr))
@@ -87,10 +86,8 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   float* qbar = reinterpret_cast<float*>(base + off_qbar);
   float* kbar = reinterpret_cast<float*>(base + off_kbar);
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(base + off_scores);
-  uint32_t* sel = reinterpret_cast<uint32_t*>(base + off_sel);
   cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, scores, s);
-  if (e == cudaSuccess) e = launch_select_topk(g, scores, sel, s);
-  if (e == cudaSuccess) e = launch_build_kv_lists(g, sel, kv_idx, kv_cnt, s);
+  if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;
 }

@@ -264,6 +264,29 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU arm
+def rank_seeds(rank, base_seeds):
+    """Weak scaling: rank r solves its own independent problems, seeds r*1000 + s."""
+    return [rank * 1000 + s for s in base_seeds]
+
+
+def reduce_over_ranks(times_ms, work, device, world):
+    """Whole-job figures: every time is the max over ranks, every amount of work
+    the sum over ranks (one all-reduce each; identity for a single rank)."""
+    import torch
+    import torch.distributed as dist
+    tot = torch.tensor(times_ms, dtype=torch.float64, device=device)
+    fl = torch.tensor(work, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
+    return tot.tolist(), fl.tolist()
+
+
+def job_value(flops, ms):
+    """TFLOP/s of `flops` done in `ms` milliseconds."""
+    return flops / (ms / 1000.0) / 1e12
+
+
 def run_gpu(args):
     import numpy as np
     import torch
@@ -286,7 +309,7 @@ def run_gpu(args):
     w = si.get_workload(args.workload)
     d = S.desc_from(w)
     plan = S.ssta_plan(d)
-    seeds = [rank * 1000 + s for s in w.seeds]
+    seeds = rank_seeds(rank, w.seeds)
     stream = torch.cuda.current_stream(dev)
 
     # per-seed resident inputs and preallocated outputs
@@ -386,15 +409,10 @@ def run_gpu(args):
     e2e_flops = flops[0][0] * args.steps
 
     # ---- reduce over ranks
-    tot = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
-    fl = torch.tensor([my_flops, my_vflops, e2e_flops], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
-    max_ms, max_e2e_ms = float(tot[0]), float(tot[1])
-    all_flops, all_vflops, all_e2e_flops = float(fl[0]), float(fl[1]), float(fl[2])
-    value = all_flops / (max_ms / 1000.0) / 1e12
-    e2e_value = all_e2e_flops / (max_e2e_ms / 1000.0) / 1e12
+    (max_ms, max_e2e_ms), (all_flops, all_vflops, all_e2e_flops) = reduce_over_ranks(
+        [elapsed_ms, e2e_ms], [my_flops, my_vflops, e2e_flops], dev, world)
+    value = job_value(all_flops, max_ms)
+    e2e_value = job_value(all_e2e_flops, max_e2e_ms)
 
     if rank == 0:
         peaks, src = load_peaks()
@@ -416,7 +434,7 @@ def run_gpu(args):
         if world == 1 and not args.no_cpu_baseline:
             xc = cpu_inputs(w, seeds[0], (0,))
             wh = si.with_overrides(w, H=1)
-            secs, f, desc = oracle_sample(wh, xc, (0,))
+            secs, f, desc = oracle_sample(wh, xc, (0,), tile_stride=12)
             cpu = {"value": f / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                    "sample": desc, "seconds": secs}
         line = {
@@ -441,7 +459,7 @@ def run_gpu(args):
             "reorder_gbs": (reorder_bytes / (reorder_ms / 1000.0) / 1e9),
             "kept_tflop_per_call": per_call_flops / 1e12,
             "valid_tflop_per_call": (my_vflops / args.steps) / 1e12,
-            "valid_tflops": all_vflops / (max_ms / 1000.0) / 1e12,
+            "valid_tflops": job_value(all_vflops, max_ms),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": max_e2e_ms / args.steps},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,

@@ -34,8 +34,12 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include "ssta_wait.cuh"
+
 namespace ssta {
 namespace {
+
+using namespace wait;
 
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
@@ -75,33 +79,8 @@ struct ChunkTables {
 };
 
 // ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
                                             uint32_t bar) {
@@ -284,38 +263,6 @@ __device__ __forceinline__ bool key_valid(const Geom& g, int t, int o) {
   return (t - g.NT) * g.N + o < g.L_text;
 }
 
-struct Ctl {
-  volatile int* abort_flag;
-  int32_t* status;
-};
-
-// Bounded wait by one thread.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*c.abort_flag) return false;
-    if (global_ns() - t0 > kTimeoutNs) {
-      *c.abort_flag = 1;
-      atomicExch(c.status, (int)SSTA_ERR_DEVICE_TIMEOUT);
-      return false;
-    }
-  }
-}
-// Bounded wait by a whole warp; the outcome is made warp-uniform.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Ctl& c) {
-  const bool ok = wait_bounded(bar, parity, c);
-  return __all_sync(0xffffffffu, ok);
-}
-// Wait used while draining after an abort: bounded, never raises the flag.
-__device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kTimeoutNs) return;
-  }
-}
-
 // ------------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(kThreads, 1)
 ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -331,7 +278,7 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
   auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffMisc + 8);
-  const Ctl ctl{abort_flag, status};
+  const Ctl ctl{abort_flag, status, kTimeoutNs};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -432,10 +379,10 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
       });
       if (n < 0) {
         // abort: let every copy this thread started land before shared memory is released
-        drain_wait(bar(BAR_Q), 0);
+        drain_wait(bar(BAR_Q), 0, kTimeoutNs);
         for (int s = 0; s < kStages; ++s) {
-          if (nK[s] > 0) drain_wait(bar(BAR_KFULL + s), (uint32_t)((nK[s] - 1) & 1));
-          if (nV[s] > 0) drain_wait(bar(BAR_VFULL + s), (uint32_t)((nV[s] - 1) & 1));
+          if (nK[s] > 0) drain_wait(bar(BAR_KFULL + s), (uint32_t)((nK[s] - 1) & 1), kTimeoutNs);
+          if (nV[s] > 0) drain_wait(bar(BAR_VFULL + s), (uint32_t)((nV[s] - 1) & 1), kTimeoutNs);
         }
       }
     }
@@ -505,7 +452,7 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
       }
       // every MMA (and its commit arrivals) retires before TMEM and smem are released
       tc_commit(bar(BAR_DRAIN));
-      drain_wait(bar(BAR_DRAIN), 0);
+      drain_wait(bar(BAR_DRAIN), 0, kTimeoutNs);
     }
   } else if (warp < 4 * nh) {
     // ------------------------------------------------------ softmax + epilogue

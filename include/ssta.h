@@ -101,7 +101,7 @@ typedef struct {
  * max_kept = NT + num_text_tiles when L_text > 0 (text query tiles attend every
  * tile), else min(NT, topk + window_tiles).
  * Returns SSTA_ERR_INVALID_ARG for malformed descriptors, SSTA_ERR_UNSUPPORTED
- * when D != 128, NT > 2048, or (bf16) N is not a multiple of 128.
+ * when D != 128, N > 4096, NT > 2048, B*H > 65535 or Lq >= 2^31.
  */
 ssta_status ssta_plan(const ssta_desc* desc, ssta_plan_info* info);
 
@@ -141,7 +141,9 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
  *   ssta_build_block_mask (read; ids must be < NQ and ascending order is not
  *   required), o_packed [B,H,Lq,D] (written, dtype), lse [B,H,Lq] fp32
  *   (written), workspace >= info.attn_workspace_bytes (device status word).
- * bf16: tcgen05 tensor-core kernel, requires N % 128 == 0.  f32: SIMT kernel.
+ * bf16: tcgen05 tensor-core kernel; needs N % 128 == 0, else
+ * SSTA_ERR_UNSUPPORTED (the paper's 4x8x8 tiles hold 256 tokens).
+ * f32: SIMT kernel, any N.
  */
 ssta_status ssta_attention_fwd(const ssta_desc* desc, const void* q_packed, const void* k_packed,
                                const void* v_packed, const int32_t* kv_idx, const int32_t* kv_cnt,
@@ -176,6 +178,18 @@ ssta_status ssta_tile_unorder(const ssta_desc* desc, const void* x_packed, void*
 #define SSTA_STATIC_SCRATCH_BYTES (32u << 20)
 ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, const void* q_packed, const void* k_packed,
                                           int32_t* kv_idx, int32_t* kv_cnt, float* tile_scores, void* stream);
+
+/*
+ * ssta_selftest_bounded_wait — runs the device-side bounded wait that guards every
+ * pipeline wait of ssta_attention_fwd on a barrier phase that never completes
+ * (complete == 0) or that completes at once (complete != 0).  The paper has no
+ * counterpart; this exists to test failure handling without faulting a GPU.
+ *   timeout_us in [1, 2,000,000]: the wait's limit; workspace >= 256 bytes.
+ * Afterwards the workspace status word (ssta_read_device_status) holds
+ * SSTA_ERR_DEVICE_TIMEOUT (never-completing phase, after about timeout_us) or 0.
+ */
+ssta_status ssta_selftest_bounded_wait(int32_t timeout_us, int32_t complete, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /*
  * ssta_read_device_status — copy the device status word (first int32 of a

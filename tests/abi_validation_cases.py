@@ -69,6 +69,11 @@ cases.append(("attn_small_workspace", attn(d, wsb=64)))
 cases.append(("attn_null_q", attn(d, q=None)))
 cases.append(("attn_misaligned_o", attn(d, o=P(A + 2))))
 cases.append(("read_status_null", call("ssta_read_device_status", None, None, None)))
+lib.ssta_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
+                                           ctypes.c_void_p]
+cases.append(("selftest_timeout_zero", lib.ssta_selftest_bounded_wait(0, 0, P(A), 4096, None)))
+cases.append(("selftest_timeout_huge", lib.ssta_selftest_bounded_wait(3000000, 0, P(A), 4096, None)))
+cases.append(("selftest_no_workspace", lib.ssta_selftest_bounded_wait(1000, 0, None, 0, None)))
 
 for name, code in cases:
     print(name, code)

@@ -11,9 +11,10 @@
 //                         valid q and k rows with 16-byte coalesced loads and
 //                         reduces per-channel fp32 sums across row groups; the
 //                         means are stored channel-major for the score kernel.
-//   tile_scores_kernel    fp32 SIMT, 128x64 score blocks per CTA, 32 channels at
-//                         a time in shared memory, channels summed in order
-//                         0..D-1 with FMA.
+//   tile_scores_kernel    fp32 SIMT, 128x128 score blocks per CTA, 8x8 per
+//                         thread, 16-channel stages double-buffered in shared
+//                         memory by cp.async, channels summed in order 0..D-1
+//                         with FMA.
 //   select_and_list_kernel one warp per (head, query tile): top-k over scores
 //                         held in registers as order-preserving 32-bit keys
 //                         (bitwise binary search for the k-th key with warp-wide
@@ -117,68 +118,119 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
   }
 }
 
-// Step 2, Score_s = Qbar Kbar^T.  One CTA computes a 128 x 64 block of scores for
-// one head; 256 threads as 16 x 16, each owning 8 rows x 4 columns.  The pooled
-// means arrive channel-major ([head][channel][tile]), so 32 channels at a time are
-// copied into shared memory with coalesced loads in the same layout, and a thread's
-// 8 + 4 operands for one channel are three 16-byte loads feeding 32 FMAs.  Every
-// score is accumulated over channels 0..D-1 in order with FMA.
-constexpr int kScoreRows = 128;
-constexpr int kScoreCols = 64;
-constexpr int kScoreChunk = 32;
+// Step 2, Score_s = Qbar Kbar^T.  One CTA computes a 128 x 128 block of scores
+// of one head with 256 threads; thread (ty, tx) of a 16 x 16 grid owns rows
+// {4ty..4ty+3, 64+4ty..64+4ty+3} and the same pattern of columns, i.e. 8 x 8
+// scores, so one channel costs it four 16-byte shared loads for 64 FMAs.  The
+// pooled means arrive channel-major ([head][channel][tile]); 16 channels of the
+// CTA's 128 query tiles and 128 key tiles form one stage, copied global ->
+// shared by cp.async (16-byte copies when NT % 4 == 0, else 4-byte ones; tiles
+// past NT are zero-filled) into two buffers, so the next stage is in flight
+// while the current one is consumed.  Every score is accumulated over channels
+// 0..D-1 in order with FMA.
+constexpr int kScoreBlock = 128;
+constexpr int kScoreStage = 16;   // channels per stage
 
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(s), "l"(gmem), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// One stage: channels d0..d0+15 of the CTA's query tiles (Qbar) and key tiles (Kbar).
+// Out-of-range tiles copy zero bytes from the head's base address (always valid).
+template <bool kVec>
+__device__ __forceinline__ void score_stage_copy(float (*qs)[kScoreBlock], float (*ks)[kScoreBlock], const float* qh,
+                                                 const float* kh, int NT, int i0, int j0, int d0) {
+  if constexpr (kVec) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = threadIdx.x + 256 * u, ch = e >> 5, r = (e & 31) * 4;
+      const bool qi = i0 + r < NT, kj = j0 + r < NT;
+      cp_async16(&qs[ch][r], qi ? qh + (int64_t)(d0 + ch) * NT + i0 + r : qh, qi);
+      cp_async16(&ks[ch][r], kj ? kh + (int64_t)(d0 + ch) * NT + j0 + r : kh, kj);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = threadIdx.x + 256 * u, ch = e >> 7, r = e & 127;
+      const bool qi = i0 + r < NT, kj = j0 + r < NT;
+      cp_async4(&qs[ch][r], qi ? qh + (int64_t)(d0 + ch) * NT + i0 + r : qh, qi);
+      cp_async4(&ks[ch][r], kj ? kh + (int64_t)(d0 + ch) * NT + j0 + r : kh, kj);
+    }
+  }
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(256, 2)
 tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __restrict__ kbar_t,
                    float* __restrict__ scores) {
-  __shared__ __align__(16) float qs[kScoreChunk][kScoreRows + 4];
-  __shared__ __align__(16) float ks[kScoreChunk][kScoreCols + 4];
+  __shared__ __align__(16) float qs[2][kScoreStage][kScoreBlock];
+  __shared__ __align__(16) float ks[2][kScoreStage][kScoreBlock];
   const int64_t bh = blockIdx.z;
-  const int i0 = blockIdx.y * kScoreRows, j0 = blockIdx.x * kScoreCols;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const float* qh = qbar_t + bh * g.D * (int64_t)g.NT;
-  const float* kh = kbar_t + bh * g.D * (int64_t)g.NT;
-  float acc[8][4];
+  const int NT = g.NT;
+  const int i0 = blockIdx.y * kScoreBlock, j0 = blockIdx.x * kScoreBlock;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const float* qh = qbar_t + bh * g.D * (int64_t)NT;
+  const float* kh = kbar_t + bh * g.D * (int64_t)NT;
+  float acc[8][8];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
 
-  for (int d0 = 0; d0 < g.D; d0 += kScoreChunk) {
-    for (int e = threadIdx.x; e < kScoreChunk * kScoreRows; e += 256) {
-      const int cc = e / kScoreRows, r = e % kScoreRows, i = i0 + r;
-      qs[cc][r] = i < g.NT ? __ldg(qh + (int64_t)(d0 + cc) * g.NT + i) : 0.f;
+  const int nst = g.D / kScoreStage;
+  score_stage_copy<kVec>(qs[0], ks[0], qh, kh, NT, i0, j0, 0);
+  cp_async_commit();
+  for (int st = 0; st < nst; ++st) {
+    const int buf = st & 1;
+    if (st + 1 < nst) {
+      // buffer buf^1 was last read in stage st-1, which every thread has left
+      score_stage_copy<kVec>(qs[buf ^ 1], ks[buf ^ 1], qh, kh, NT, i0, j0, (st + 1) * kScoreStage);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    for (int e = threadIdx.x; e < kScoreChunk * kScoreCols; e += 256) {
-      const int cc = e / kScoreCols, r = e % kScoreCols, j = j0 + r;
-      ks[cc][r] = j < g.NT ? __ldg(kh + (int64_t)(d0 + cc) * g.NT + j) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int cc = 0; cc < kScoreChunk; ++cc) {
-      const float4 qa = *reinterpret_cast<const float4*>(&qs[cc][ty * 8]);
-      const float4 qb = *reinterpret_cast<const float4*>(&qs[cc][ty * 8 + 4]);
-      const float4 kv = *reinterpret_cast<const float4*>(&ks[cc][tx * 4]);
+    __syncthreads();   // stage st visible to every thread
+#pragma unroll
+    for (int c = 0; c < kScoreStage; ++c) {
+      const float4 qa = *reinterpret_cast<const float4*>(&qs[buf][c][4 * ty]);
+      const float4 qb = *reinterpret_cast<const float4*>(&qs[buf][c][64 + 4 * ty]);
+      const float4 ka = *reinterpret_cast<const float4*>(&ks[buf][c][4 * tx]);
+      const float4 kb = *reinterpret_cast<const float4*>(&ks[buf][c][64 + 4 * tx]);
       const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-      const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+      const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], kk[b], acc[a][b]);
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
     }
-    __syncthreads();
+    __syncthreads();   // every thread is done with buffer buf before it is refilled
   }
-  float* sh = scores + bh * g.NT * (int64_t)g.NT;
+  float* sh = scores + bh * NT * (int64_t)NT;
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
-    const int i = i0 + ty * 8 + a;
-    if (i >= g.NT) continue;
-    const int j = j0 + tx * 4;
-    if (j + 3 < g.NT && (g.NT % 4) == 0) {
-      *reinterpret_cast<float4*>(sh + (int64_t)i * g.NT + j) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-    } else {
+    const int i = i0 + (a < 4 ? 4 * ty + a : 64 + 4 * ty + a - 4);
+    if (i >= NT) continue;
+    float* srow = sh + (int64_t)i * NT;
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
-        if (j + b < g.NT) sh[(int64_t)i * g.NT + j + b] = acc[a][b];
+    for (int half = 0; half < 2; ++half) {
+      const int j = j0 + 64 * half + 4 * tx;
+      const float* v = &acc[a][4 * half];
+      if constexpr (kVec) {
+        if (j < NT) *reinterpret_cast<float4*>(srow + j) = make_float4(v[0], v[1], v[2], v[3]);
+      } else {
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          if (j + b < NT) srow[j + b] = v[b];
+      }
     }
   }
 }
@@ -395,8 +447,11 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
                                cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
-  dim3 grid(ceil_div(g.NT, kScoreCols), ceil_div(g.NT, kScoreRows), g.B * g.H);
-  tile_scores_kernel<<<grid, 256, 0, s>>>(g, qbar, kbar, scores);
+  dim3 grid(ceil_div(g.NT, kScoreBlock), ceil_div(g.NT, kScoreBlock), g.B * g.H);
+  if (g.NT % 4 == 0)
+    tile_scores_kernel<true><<<grid, 256, 0, s>>>(g, qbar, kbar, scores);
+  else
+    tile_scores_kernel<false><<<grid, 256, 0, s>>>(g, qbar, kbar, scores);
   return cudaGetLastError();
 }
 

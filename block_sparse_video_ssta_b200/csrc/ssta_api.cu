@@ -131,12 +131,12 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
     return SSTA_ERR_ALIGNMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  if (cudaMemsetAsync(w + ws.status, 0, sizeof(int32_t), s) != cudaSuccess) return SSTA_ERR_LAUNCH;
-  if (empty) return SSTA_OK;
+  if (empty) return from_cuda(cudaMemsetAsync(w + ws.status, 0, sizeof(int32_t), s));
   float* qbar = reinterpret_cast<float*>(w + ws.qbar);
   float* kbar = reinterpret_cast<float*>(w + ws.kbar);
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(w + ws.scores);
-  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, s);
+  // the pool kernel also clears the status word
+  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(w + ws.status), s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return from_cuda(e);

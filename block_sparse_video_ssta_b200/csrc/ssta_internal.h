@@ -49,8 +49,10 @@ cudaError_t launch_tile_reorder(const Geom& g, const void* raster, const void* t
                                 cudaStream_t s);
 cudaError_t launch_tile_unorder(const Geom& g, const void* packed, void* raster, void* text,
                                 cudaStream_t s);
+// Also writes 0 to *status (when non-NULL) after the previous kernel of the stream has
+// finished, so a mask build needs no separate reset of its status word.
 cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, float* qbar, float* kbar,
-                             cudaStream_t s);
+                             int32_t* status, cudaStream_t s);
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
                                cudaStream_t s);
 cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,

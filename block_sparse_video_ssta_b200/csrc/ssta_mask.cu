@@ -14,7 +14,7 @@
 //   tile_scores_kernel    fp32 SIMT, 128x128 score blocks per CTA, 8x8 per
 //                         thread, 16-channel stages double-buffered in shared
 //                         memory by cp.async, channels summed in order 0..D-1
-//                         with FMA.
+//                         with FMA (packed f32x2, two columns per instruction).
 //   select_and_list_kernel one warp per (head, query tile): top-k over scores
 //                         held in registers as order-preserving 32-bit keys
 //                         (bitwise binary search for the k-th key with warp-wide
@@ -28,6 +28,29 @@
 
 namespace ssta {
 namespace {
+
+// Programmatic dependent launch: a kernel launched with launch_dependent() may start
+// while the previous kernel of the stream is still running; grid_dependency_wait()
+// blocks until that kernel has completed and its writes are visible, and
+// allow_dependents() lets the next kernel start launching.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 constexpr int kPoolThreads = 256;
 
@@ -51,7 +74,10 @@ __device__ __forceinline__ void add_vec(float* acc, const int4& raw, const float
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ kp,
-                 float* __restrict__ qbar, float* __restrict__ kbar) {
+                 float* __restrict__ qbar, float* __restrict__ kbar, int32_t* __restrict__ status) {
+  allow_dependents();
+  grid_dependency_wait();   // q and k are packed by the previous kernels
+  if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
   constexpr int EPV = 16 / sizeof(T);        // elements per 16-byte vector
   const int vpr = g.D / EPV;                 // vectors per row
   const int rpp = kPoolThreads / vpr;        // rows per pass
@@ -127,7 +153,23 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
 // shared by cp.async (16-byte copies when NT % 4 == 0, else 4-byte ones; tiles
 // past NT are zero-filled) into two buffers, so the next stage is in flight
 // while the current one is consumed.  Every score is accumulated over channels
-// 0..D-1 in order with FMA.
+// 0..D-1 in order with FMA, two adjacent columns per fma.rn.f32x2 instruction.
+// Two-lane fp32 arithmetic (sm_100): one instruction for a pair of values, each
+// lane rounded exactly as the scalar instruction would.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 constexpr int kScoreBlock = 128;
 constexpr int kScoreStage = 16;   // channels per stage
 
@@ -179,13 +221,15 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const float* qh = qbar_t + bh * g.D * (int64_t)NT;
   const float* kh = kbar_t + bh * g.D * (int64_t)NT;
-  float acc[8][8];
+  uint64_t acc[8][4];   // pairs of adjacent columns (f32x2)
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0ull;
 
   const int nst = g.D / kScoreStage;
+  allow_dependents();
+  grid_dependency_wait();   // the pooled means are written by the previous kernel
   score_stage_copy<kVec>(qs[0], ks[0], qh, kh, NT, i0, j0, 0);
   cp_async_commit();
   for (int st = 0; st < nst; ++st) {
@@ -206,11 +250,13 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
       const float4 ka = *reinterpret_cast<const float4*>(&ks[buf][c][4 * tx]);
       const float4 kb = *reinterpret_cast<const float4*>(&ks[buf][c][64 + 4 * tx]);
       const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-      const float kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      const uint64_t k2[4] = {f2_pack(ka.x, ka.y), f2_pack(ka.z, ka.w), f2_pack(kb.x, kb.y), f2_pack(kb.z, kb.w)};
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
+      for (int a = 0; a < 8; ++a) {
+        const uint64_t q2 = f2_pack(qv[a], qv[a]);
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
+        for (int b = 0; b < 4; ++b) acc[a][b] = f2_fma(q2, k2[b], acc[a][b]);
+      }
     }
     __syncthreads();   // every thread is done with buffer buf before it is refilled
   }
@@ -223,7 +269,9 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int j = j0 + 64 * half + 4 * tx;
-      const float* v = &acc[a][4 * half];
+      float v[4];
+      f2_unpack(acc[a][2 * half], v[0], v[1]);
+      f2_unpack(acc[a][2 * half + 1], v[2], v[3]);
       if constexpr (kVec) {
         if (j < NT) *reinterpret_cast<float4*>(srow + j) = make_float4(v[0], v[1], v[2], v[3]);
       } else {
@@ -271,6 +319,7 @@ __device__ __forceinline__ uint32_t range_bits(int word, int lo, int hi) {
 //    32-tile words, followed by the text tiles and -1 padding.
 // Text query tiles keep every tile.
 constexpr int kBucketCap = 64;
+constexpr int kHiBits = 12;   // prefix bits searched over every key
 
 template <int SLOTS>
 __global__ void __launch_bounds__(256)
@@ -280,6 +329,7 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // bh * NQ + i
   if (row >= (int64_t)g.B * g.H * g.NQ) return;
+  grid_dependency_wait();   // the scores are written by the previous kernel
   const int64_t bh = row / g.NQ;
   const int i = (int)(row - bh * g.NQ);
   int32_t* out = kv_idx + row * g.max_kept;
@@ -299,44 +349,51 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
     for (int q = 0; q < (SLOTS + 31) / 32; ++q) myword[q] = 0u;
     const int k = g.k;
     if (k > 0) {
-      // k-th largest key in two levels: a bitwise search over the upper 16 bits of every
-      // key, then over the lower 16 bits of the keys that share the found upper half
-      // (the boundary bucket, compacted into shared memory when it holds at most 64;
-      // otherwise the lower bits are searched over all keys).
+      // k-th largest key in two levels: a bitwise search over the upper kHiBits bits of
+      // every key, then over the remaining low bits of the keys that share the found
+      // prefix (the boundary bucket, compacted into shared memory when it holds at most
+      // 64; otherwise the low bits are searched over all keys).  `above` = number of
+      // keys whose prefix is larger, i.e. the count of the last candidate that failed.
+      constexpr int kLoBits = 32 - kHiBits;
       uint32_t hi = 0;
-      for (int bit = 15; bit >= 0; --bit) {
-        const uint32_t cand = (hi | (1u << bit)) << 16;
-        int cnt = 0;
+      int above = 0;
+      for (int bit = kHiBits - 1; bit >= 0; --bit) {
+        const uint32_t cand = (hi | (1u << bit)) << kLoBits;
+        int c0 = 0, c1 = 0;
 #pragma unroll
-        for (int w = 0; w < SLOTS; ++w) cnt += (key[w] >= cand) ? 1 : 0;
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        for (int w = 0; w < SLOTS; w += 2) {
+          c0 += (key[w] >= cand) ? 1 : 0;
+          if (w + 1 < SLOTS) c1 += (key[w + 1] >= cand) ? 1 : 0;
+        }
+        const int cnt = __reduce_add_sync(0xffffffffu, c0 + c1);
         if (cnt >= k) hi |= 1u << bit;
+        else above = cnt;
       }
-      int above = 0, bsize = 0;
+      int bsize = 0;
       uint32_t* bucket = bucket_smem + (threadIdx.x >> 5) * kBucketCap;
 #pragma unroll
       for (int w = 0; w < SLOTS; ++w) {
-        above += ((key[w] >> 16) > hi) ? 1 : 0;
-        const bool in = key[w] != 0u && (key[w] >> 16) == hi;
+        const bool in = key[w] != 0u && (key[w] >> kLoBits) == hi;
         const uint32_t m = __ballot_sync(0xffffffffu, in);
-        const int pos = bsize + __popc(m & lt_mask);
-        if (in && pos < kBucketCap) bucket[pos] = key[w];
-        bsize += __popc(m);
+        if (m) {   // warp-uniform; most slots hold no key of the bucket
+          const int pos = bsize + __popc(m & lt_mask);
+          if (in && pos < kBucketCap) bucket[pos] = key[w];
+          bsize += __popc(m);
+        }
       }
-      above = __reduce_add_sync(0xffffffffu, above);
       __syncwarp();
       const int need_lo = k - above;     // keys to take from the bucket (>= 1)
-      uint32_t thr = hi << 16;
+      uint32_t thr = hi << kLoBits;
       if (bsize <= kBucketCap) {
         const uint32_t b0 = lane < bsize ? bucket[lane] : 0u;
         const uint32_t b1 = lane + 32 < bsize ? bucket[lane + 32] : 0u;
-        for (int bit = 15; bit >= 0; --bit) {
+        for (int bit = kLoBits - 1; bit >= 0; --bit) {
           const uint32_t cand = thr | (1u << bit);
           const int cnt = __reduce_add_sync(0xffffffffu, (b0 >= cand ? 1 : 0) + (b1 >= cand ? 1 : 0));
           if (cnt >= need_lo) thr = cand;
         }
       } else {
-        for (int bit = 15; bit >= 0; --bit) {
+        for (int bit = kLoBits - 1; bit >= 0; --bit) {
           const uint32_t cand = thr | (1u << bit);
           int cnt = 0;
 #pragma unroll
@@ -346,21 +403,34 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
         }
       }
       __syncwarp();
-      int gt = 0;
+      // keys above the k-th key, and keys equal to it (16-bit fields of one count)
+      uint32_t gt_ge = 0;
 #pragma unroll
-      for (int w = 0; w < SLOTS; ++w) gt += (key[w] > thr) ? 1 : 0;
-      gt = __reduce_add_sync(0xffffffffu, gt);
+      for (int w = 0; w < SLOTS; ++w) gt_ge += (key[w] > thr ? 1u : 0u) + (key[w] >= thr ? 0x10000u : 0u);
+      gt_ge = __reduce_add_sync(0xffffffffu, gt_ge);
+      const int gt = (int)(gt_ge & 0xffffu), ge = (int)(gt_ge >> 16);
       const int need = k - gt;
-      int eq_before = 0;
+      if (ge == k) {
+        // every key equal to the k-th is taken: no tie to break
 #pragma unroll
-      for (int w = 0; w < SLOTS; ++w) {
-        if (w < g.words) {
-          const bool eq = key[w] == thr;
-          const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-          const bool take = key[w] > thr || (eq && eq_before + __popc(eqm & lt_mask) < need);
-          const uint32_t word = __ballot_sync(0xffffffffu, take);
-          if ((w & 31) == lane) myword[w >> 5] = word;
-          eq_before += __popc(eqm);
+        for (int w = 0; w < SLOTS; ++w) {
+          if (w < g.words) {
+            const uint32_t word = __ballot_sync(0xffffffffu, key[w] >= thr);
+            if ((w & 31) == lane) myword[w >> 5] = word;
+          }
+        }
+      } else {
+        int eq_before = 0;
+#pragma unroll
+        for (int w = 0; w < SLOTS; ++w) {
+          if (w < g.words) {
+            const bool eq = key[w] == thr;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool take = key[w] > thr || (eq && eq_before + __popc(eqm & lt_mask) < need);
+            const uint32_t word = __ballot_sync(0xffffffffu, take);
+            if ((w & 31) == lane) myword[w >> 5] = word;
+            eq_before += __popc(eqm);
+          }
         }
       }
     }
@@ -429,19 +499,19 @@ MaskWorkspace mask_workspace_layout(const Geom& g) {
 }
 
 cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, float* qbar, float* kbar,
-                             cudaStream_t s) {
+                             int32_t* status, cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
   dim3 grid(g.NT, g.B * g.H);
   const int epv = 16 / g.esize;
   const int rpp = kPoolThreads / (g.D / epv);
   const size_t smem = 2 * rpp * g.D * sizeof(float);
+  const int4* q4 = static_cast<const int4*>(qp);
+  const int4* k4 = static_cast<const int4*>(kp);
   if (g.dtype == SSTA_BF16)
-    tile_pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, smem, s>>>(
-        g, static_cast<const int4*>(qp), static_cast<const int4*>(kp), qbar, kbar);
-  else
-    tile_pool_kernel<float><<<grid, kPoolThreads, smem, s>>>(
-        g, static_cast<const int4*>(qp), static_cast<const int4*>(kp), qbar, kbar);
-  return cudaGetLastError();
+    return launch_dependent(tile_pool_kernel<__nv_bfloat16>, grid, dim3(kPoolThreads), smem, s, g, q4, k4, qbar,
+                            kbar, status);
+  return launch_dependent(tile_pool_kernel<float>, grid, dim3(kPoolThreads), smem, s, g, q4, k4, qbar, kbar,
+                          status);
 }
 
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
@@ -449,10 +519,8 @@ cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kb
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
   dim3 grid(ceil_div(g.NT, kScoreBlock), ceil_div(g.NT, kScoreBlock), g.B * g.H);
   if (g.NT % 4 == 0)
-    tile_scores_kernel<true><<<grid, 256, 0, s>>>(g, qbar, kbar, scores);
-  else
-    tile_scores_kernel<false><<<grid, 256, 0, s>>>(g, qbar, kbar, scores);
-  return cudaGetLastError();
+    return launch_dependent(tile_scores_kernel<true>, grid, dim3(256), 0, s, g, qbar, kbar, scores);
+  return launch_dependent(tile_scores_kernel<false>, grid, dim3(256), 0, s, g, qbar, kbar, scores);
 }
 
 cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
@@ -460,15 +528,10 @@ cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* 
   const int64_t rows = (int64_t)g.B * g.H * g.NQ;
   if (rows == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((rows + 7) / 8);
-  if (g.words <= 8)
-    select_and_list_kernel<8><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
-  else if (g.words <= 16)
-    select_and_list_kernel<16><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
-  else if (g.words <= 32)
-    select_and_list_kernel<32><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
-  else
-    select_and_list_kernel<64><<<blocks, 256, 0, s>>>(g, scores, kv_idx, kv_cnt);
-  return cudaGetLastError();
+  if (g.words <= 8) return launch_dependent(select_and_list_kernel<8>, dim3(blocks), dim3(256), 0, s, g, scores, kv_idx, kv_cnt);
+  if (g.words <= 16) return launch_dependent(select_and_list_kernel<16>, dim3(blocks), dim3(256), 0, s, g, scores, kv_idx, kv_cnt);
+  if (g.words <= 32) return launch_dependent(select_and_list_kernel<32>, dim3(blocks), dim3(256), 0, s, g, scores, kv_idx, kv_cnt);
+  return launch_dependent(select_and_list_kernel<64>, dim3(blocks), dim3(256), 0, s, g, scores, kv_idx, kv_cnt);
 }
 
 }  // namespace ssta

@@ -81,12 +81,12 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   if (st != SSTA_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(base_v);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(base, 0, sizeof(int32_t), s) != cudaSuccess) return SSTA_ERR_LAUNCH;
-  if (empty) return SSTA_OK;
+  if (empty) return cudaMemsetAsync(base, 0, sizeof(int32_t), s) == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;
   float* qbar = reinterpret_cast<float*>(base + off_qbar);
   float* kbar = reinterpret_cast<float*>(base + off_kbar);
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(base + off_scores);
-  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, s);
+  // the pool kernel also clears the status word
+  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(base), s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;

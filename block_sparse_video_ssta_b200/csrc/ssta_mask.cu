@@ -98,15 +98,15 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
 
   if (full) {
     int o = rsub;
-    for (; o + 3 * rpp < g.N; o += 4 * rpp) {
-      int4 rq[4], rk[4];
+    for (; o + 7 * rpp < g.N; o += 8 * rpp) {
+      int4 rq[8], rk[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         rq[u] = __ldg(qp + base + (int64_t)(o + u * rpp) * vpr);
         rk[u] = __ldg(kp + base + (int64_t)(o + u * rpp) * vpr);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         add_vec(aq, rq[u], (const T*)nullptr);
         add_vec(ak, rk[u], (const T*)nullptr);
       }

@@ -125,6 +125,17 @@ def test_full_size_sampled(cuda_ok, name):
     assert st["rows_mask_mismatch"] <= max(2, g.NT // 100)
 
 
+def test_more_than_1024_tiles(cuda_ok):
+    """NT = 1,056 video tiles (4 x 264 x 256 grid, 4x8x8 tiles): the widest selection
+    instance (up to 2,048 tiles per row), checked on every mask row and on sampled tiles."""
+    w = with_overrides(si.get_workload("small_bf16"), H=1, T=4, Y=264, X=256, topk=40, wT=1, wY=3, wX=3)
+    g = oracle.geometry(w)
+    assert g.NT == 1056
+    st = full_check(w, seed=2, q_tiles=_sampled(w, stride=64))
+    _report("NT=1056", st)
+    assert st["rows_mask_mismatch"] <= 2
+
+
 def test_deterministic_masks_and_outputs(cuda_ok):
     w = si.get_workload("small_bf16")
     x = si.make_inputs(w, 1, device="cuda")

@@ -125,7 +125,7 @@ class Plan:
 
 def ssta_plan(desc: Desc) -> Plan:
     info = _PlanInfo()
-    _check(lib.ssta_plan(ctypes.byref(desc), ctypes.byref(info)), "ssta_plan")
+    _call("ssta_plan", None, ctypes.byref(desc), ctypes.byref(info))
     return Plan(*(getattr(info, f[0]) for f in _PlanInfo._fields_))
 
 
@@ -157,6 +157,16 @@ def _ptr(t, name, dtype=None, shape=None, optional=False):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _call(name, dev, *args):
+    """Call C-ABI function `name` with CUDA device `dev` current (the device whose stream
+    and tensors the call receives; None for host-only calls); raise on a non-zero status."""
+    fn = getattr(lib, name)
+    if dev is None:
+        return _check(fn(*args), name)
+    with torch.cuda.device(dev):
+        return _check(fn(*args), name)
+
+
 def _workspace(nbytes, device):
     # 256-byte aligned (the caching allocator returns 512-byte aligned blocks)
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
@@ -169,12 +179,12 @@ def ssta_tile_reorder(desc: Desc, x_raster, x_text=None, x_packed=None, stream=N
     dev = x_raster.device
     if x_packed is None:
         x_packed = torch.empty((desc.B, desc.H, p.packed_len, desc.D), dtype=dt, device=dev)
-    _check(lib.ssta_tile_reorder(
-        ctypes.byref(desc),
+    _call(
+        "ssta_tile_reorder", dev, ctypes.byref(desc),
         _ptr(x_raster, "x_raster", dt, (desc.B, desc.H, desc.T, desc.Y, desc.X, desc.D)),
         _ptr(x_text, "x_text", dt, (desc.B, desc.H, desc.L_text, desc.D), optional=desc.L_text == 0),
         _ptr(x_packed, "x_packed", dt, (desc.B, desc.H, p.packed_len, desc.D)),
-        _stream(stream, dev)), "ssta_tile_reorder")
+        _stream(stream, dev))
     return x_packed
 
 
@@ -191,13 +201,14 @@ def ssta_build_block_mask(desc: Desc, q_packed, k_packed, kv_idx=None, kv_cnt=No
         kv_cnt = torch.empty((desc.B, desc.H, p.num_q_tiles), dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = _workspace(p.workspace_bytes, dev)
-    _check(lib.ssta_build_block_mask(
-        ctypes.byref(desc), _ptr(q_packed, "q_packed", dt, shp), _ptr(k_packed, "k_packed", dt, shp),
+    _call(
+        "ssta_build_block_mask", dev, ctypes.byref(desc),
+        _ptr(q_packed, "q_packed", dt, shp), _ptr(k_packed, "k_packed", dt, shp),
         _ptr(kv_idx, "kv_idx", torch.int32, (desc.B, desc.H, p.num_q_tiles, p.max_kept)),
         _ptr(kv_cnt, "kv_cnt", torch.int32, (desc.B, desc.H, p.num_q_tiles)),
         _ptr(tile_scores, "tile_scores", torch.float32, (desc.B, desc.H, p.num_tiles, p.num_tiles), optional=True),
         _ptr(workspace, "workspace", torch.uint8), ctypes.c_size_t(workspace.numel()),
-        _stream(stream, dev)), "ssta_build_block_mask")
+        _stream(stream, dev))
     return kv_idx, kv_cnt, workspace
 
 
@@ -214,14 +225,15 @@ def ssta_attention_fwd(desc: Desc, q_packed, k_packed, v_packed, kv_idx, kv_cnt,
         lse = torch.empty((desc.B, desc.H, p.packed_len), dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = _workspace(p.attn_workspace_bytes, dev)
-    _check(lib.ssta_attention_fwd(
-        ctypes.byref(desc), _ptr(q_packed, "q_packed", dt, shp), _ptr(k_packed, "k_packed", dt, shp),
+    _call(
+        "ssta_attention_fwd", dev, ctypes.byref(desc),
+        _ptr(q_packed, "q_packed", dt, shp), _ptr(k_packed, "k_packed", dt, shp),
         _ptr(v_packed, "v_packed", dt, shp),
         _ptr(kv_idx, "kv_idx", torch.int32, (desc.B, desc.H, p.num_q_tiles, p.max_kept)),
         _ptr(kv_cnt, "kv_cnt", torch.int32, (desc.B, desc.H, p.num_q_tiles)),
         _ptr(o_packed, "o_packed", dt, shp), _ptr(lse, "lse", torch.float32, shp[:3]),
         _ptr(workspace, "workspace", torch.uint8), ctypes.c_size_t(workspace.numel()),
-        _stream(stream, dev)), "ssta_attention_fwd")
+        _stream(stream, dev))
     return o_packed, lse, workspace
 
 
@@ -234,20 +246,20 @@ def ssta_tile_unorder(desc: Desc, x_packed, x_raster=None, x_text=None, stream=N
         x_raster = torch.empty((desc.B, desc.H, desc.T, desc.Y, desc.X, desc.D), dtype=dt, device=dev)
     if x_text is None and want_text and desc.L_text > 0:
         x_text = torch.empty((desc.B, desc.H, desc.L_text, desc.D), dtype=dt, device=dev)
-    _check(lib.ssta_tile_unorder(
-        ctypes.byref(desc), _ptr(x_packed, "x_packed", dt, (desc.B, desc.H, p.packed_len, desc.D)),
+    _call(
+        "ssta_tile_unorder", dev, ctypes.byref(desc),
+        _ptr(x_packed, "x_packed", dt, (desc.B, desc.H, p.packed_len, desc.D)),
         _ptr(x_raster, "x_raster", dt, (desc.B, desc.H, desc.T, desc.Y, desc.X, desc.D)),
         _ptr(x_text, "x_text", dt, (desc.B, desc.H, desc.L_text, desc.D), optional=True),
-        _stream(stream, dev)), "ssta_tile_unorder")
+        _stream(stream, dev))
     return x_raster, x_text
 
 
 def ssta_read_device_status(workspace, stream=None) -> int:
     """Device status word of a workspace (0 = no device-side error).  Synchronises the stream."""
     code = ctypes.c_int32(-1)
-    _check(lib.ssta_read_device_status(_ptr(workspace, "workspace", torch.uint8),
-                                       _stream(stream, workspace.device), ctypes.byref(code)),
-           "ssta_read_device_status")
+    _call("ssta_read_device_status", workspace.device, _ptr(workspace, "workspace", torch.uint8),
+          _stream(stream, workspace.device), ctypes.byref(code))
     return int(code.value)
 
 

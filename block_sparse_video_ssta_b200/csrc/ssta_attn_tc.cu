@@ -34,6 +34,8 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "ssta_wait.cuh"
 
 namespace ssta {
@@ -58,6 +60,7 @@ constexpr uint32_t kSmemUsed = kOffMisc + 64;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // slack to align the base to 1024 B
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 1500000000ull;      // 1.5 s per wait
+constexpr int kMaxDevices = 64;
 
 enum : int {
   BAR_Q = 0, BAR_KFULL = 1, BAR_KEMPTY = 3, BAR_VFULL = 5, BAR_VEMPTY = 7,
@@ -629,12 +632,16 @@ cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* 
   if (BH == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qp, g) || !make_map(&mk, kp, g) || !make_map(&mv, vp, g)) return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ssta_attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemAlloc);
+  // the shared-memory opt-in is a per-device attribute of the kernel: set it once per device
+  static std::atomic<bool> attr_set[kMaxDevices];
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(ssta_attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int bands = (g.N + 255) / 256;
   const int64_t units = BH * (int64_t)g.NQ * bands;

@@ -16,7 +16,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_functions():
-    text = open(os.path.join(ROOT, "include", "ssta.h")).read()
+    with open(os.path.join(ROOT, "include", "ssta.h")) as f:
+        text = f.read()
     return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+(ssta_\w+)\s*\(", text, flags=re.M)))
 
 

@@ -41,7 +41,7 @@ def _rank(rank, world, port, out):
 
 def test_two_rank_reduction_and_sharding():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_rank, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)

@@ -11,7 +11,9 @@ GOLD = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_
 
 def load_golden():
     kept, lse, o = {}, {}, {}
-    for line in open(GOLD):
+    with open(GOLD) as f:
+        lines = f.read().splitlines()
+    for line in lines:
         if line.startswith("#") or not line.strip():
             continue
         parts = line.split()

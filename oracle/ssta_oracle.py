@@ -21,14 +21,26 @@ the method states it.  Sources (page titles; sections / equations named):
       doubts the AND of Algorithm 1 and points to a union; the union is used).
 * "HunyuanVideo-1.5: An 8.3B-Parameter Video Diffusion Model Built for
   Consumer GPUs" (apoapsis blog), "Under the Hood: SSTA and Muon in Detail":
-  top-k is clamped to the number of key blocks.
+  top-k is clamped to the number of key blocks; the importance-sampling
+  routine (pooled q and k normalised to unit length; similarity and key-key
+  terms mapped by (x + 1) / 2; the key-key diagonal excluded from the mean;
+  score = lambda * similarity - (1 - lambda) * redundancy, lambda = 0.9).
+
+Modes (descriptor fields, defaults first): ``score_mode`` "similarity" (raw
+pooled dot product) or "importance" (Step 2's similarity-minus-redundancy
+score in the blog's normalised form, weight ``lam``); ``combine`` "union" or
+"and" (Algorithm 1's literal M_sel AND M_sta); ``window_mode`` "shift" (the
+window slides inward at grid edges) or "truncate" (the window is cut at the
+edges, the plain reading of "within +-w/2").
 
 Readings where the pages leave a step open (each also listed in the design
-notes): similarity scores are the raw dot product of per-tile means of q and k
-over the tile's valid tokens (no normalisation, no redundancy term); the
-top-k decision is taken on the scores rounded to float32 with ties going to
-the lower tile index; the window slides inward at grid edges so it always
-keeps min(w, n) tiles per axis; selection and window are united; an optional
+notes): by default, similarity scores are the raw dot product of per-tile means
+of q and k over the tile's valid tokens (no normalisation, no redundancy term);
+in importance mode an all-zero pooled vector stays zero when normalised and a
+grid of one tile has redundancy 0; the top-k decision is taken on the scores rounded to float32 with ties going to
+the lower tile index; by default the window slides inward at grid edges so it
+always keeps min(w, n) tiles per axis, and selection and window are united; an
+optional
 text segment is appended after the video tiles, attended densely by every
 query and whose queries attend every valid key; pad tokens (grid rounded up to
 whole tiles) are never attended; LSE is the natural-log sum of exponentials of
@@ -47,7 +59,7 @@ import numpy as np
 
 __all__ = [
     "Geometry", "geometry", "valid_token_mask", "tile_reorder", "tile_unorder",
-    "tile_pool", "tile_scores", "select_topk", "window_mask", "kept_mask",
+    "tile_pool", "tile_scores", "importance_scores", "block_scores", "select_topk", "window_mask", "kept_mask",
     "kept_lists", "attention", "ssta_forward", "attention_flops",
 ]
 
@@ -164,6 +176,41 @@ def tile_scores(d, qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
     return np.einsum("bhid,bhjd->bhij", qbar, kbar)
 
 
+def _unit(x: np.ndarray) -> np.ndarray:
+    """Rows of x scaled to unit L2 length over the last axis; an all-zero row stays zero."""
+    n = np.sqrt((x * x).sum(axis=-1, keepdims=True))
+    return np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0)
+
+
+def importance_scores(d, qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """Step 2 with the redundancy term ("Selective Mask Generation": Score_i =
+    lambda Score_s - beta Score_r, Score_r the mean key-key similarity of a key
+    block to the other key blocks), in the blog's importance-sampling form:
+    pooled q and k normalised to unit length, similarity (q.k + 1) / 2 and
+    key-key similarity (k.k' + 1) / 2, the redundancy of key tile j the mean of
+    the key-key similarities of j with every other key tile (diagonal
+    excluded; 0 when there is no other tile), score = lam * similarity -
+    (1 - lam) * redundancy.  float64 [B,H,NT,NT]."""
+    lam = float(getattr(d, "lam", 0.9))
+    qn, kn = _unit(qbar), _unit(kbar)
+    sim = (np.einsum("bhid,bhjd->bhij", qn, kn) + 1.0) / 2.0
+    kk = (np.einsum("bhad,bhjd->bhaj", kn, kn) + 1.0) / 2.0      # [.., a, j]: key a vs key j
+    NT = kk.shape[-1]
+    off = ~np.eye(NT, dtype=bool)
+    if NT > 1:
+        red = (kk * off).sum(axis=-2) / (NT - 1)                # mean over a != j
+    else:
+        red = np.zeros(kk.shape[:-2] + (NT,))
+    return lam * sim - (1.0 - lam) * red[..., None, :]
+
+
+def block_scores(d, qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """The block score that Topk ranks, per the descriptor's ``score_mode``."""
+    if getattr(d, "score_mode", "similarity") == "importance":
+        return importance_scores(d, qbar, kbar)
+    return tile_scores(d, qbar, kbar)
+
+
 def select_topk(d, scores: np.ndarray) -> np.ndarray:
     """Step 2, Topk + Indexes2mask: bool [B,H,NT,NT], True where key tile j is selected for query tile i.
 
@@ -179,34 +226,42 @@ def select_topk(d, scores: np.ndarray) -> np.ndarray:
     return sel
 
 
-def _axis_window(n: int, w: int) -> np.ndarray:
-    """bool[n, n]: per-axis window membership, sliding inward at the edges."""
+def _axis_window(n: int, w: int, truncate: bool = False) -> np.ndarray:
+    """bool[n, n]: per-axis window membership.  The window of tile c covers
+    [c - w//2, c - w//2 + w); "shift" slides it inward at the edges so it keeps
+    min(w, n) tiles, "truncate" cuts it at 0 and n."""
     m = np.zeros((n, n), dtype=bool)
     span = min(w, n)
     for c in range(n):
-        start = min(max(c - w // 2, 0), n - span)
-        m[c, start: start + span] = True
+        if truncate:
+            lo = c - w // 2
+            m[c, max(lo, 0): min(lo + w, n)] = True
+        else:
+            start = min(max(c - w // 2, 0), n - span)
+            m[c, start: start + span] = True
     return m
 
 
 def window_mask(d) -> np.ndarray:
     """Step 3, M_sta: bool [NT, NT] (head-agnostic), product of the three per-axis windows."""
     g = geometry(d)
-    mt, my, mx = _axis_window(g.nT, d.wT), _axis_window(g.nY, d.wY), _axis_window(g.nX, d.wX)
+    tr = getattr(d, "window_mode", "shift") == "truncate"
+    mt, my, mx = _axis_window(g.nT, d.wT, tr), _axis_window(g.nY, d.wY, tr), _axis_window(g.nX, d.wX, tr)
     m = mt[:, None, None, :, None, None] & my[None, :, None, None, :, None] & mx[None, None, :, None, None, :]
     return m.reshape(g.NT, g.NT)
 
 
 def kept_mask(d, sel: np.ndarray) -> np.ndarray:
-    """Step 4, combined mask as a union: bool [B,H,NQ,NT+n_text].
+    """Step 4, combined mask: bool [B,H,NQ,NT+n_text].
 
-    Video query tiles keep selected | window | every text tile; text query
-    tiles keep every tile.
+    Video query tiles keep (selected | window), or (selected & window) with
+    ``combine`` = "and", plus every text tile; text query tiles keep every tile.
     """
     g = geometry(d)
     B, H = sel.shape[:2]
     kept = np.zeros((B, H, g.NQ, g.NT + g.n_text), dtype=bool)
-    kept[:, :, : g.NT, : g.NT] = sel | window_mask(d)[None, None]
+    win = window_mask(d)[None, None]
+    kept[:, :, : g.NT, : g.NT] = (sel & win) if getattr(d, "combine", "union") == "and" else (sel | win)
     kept[:, :, : g.NT, g.NT:] = True
     kept[:, :, g.NT:, :] = True
     return kept
@@ -235,7 +290,9 @@ def attention(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, kept: np.ndarra
     the valid keys j of the kept tiles of i (full attention inside each kept
     tile), LSE = log sum_j exp(s_j), O = sum_j exp(s_j - LSE) v_j.  Returns
     (O [B,H,Lq,D], LSE [B,H,Lq]); rows of tiles not in ``q_tiles`` (default:
-    all) are NaN.
+    all) are NaN.  A query tile with no kept valid key (possible with
+    ``combine`` = "and" and no text) gets O = 0 and LSE = -inf (the sum over an
+    empty set).
     """
     g = geometry(d)
     scale = 1.0 / math.sqrt(g.D) if not scale else scale
@@ -255,7 +312,11 @@ def attention(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, kept: np.ndarra
                 for j in np.nonzero(kept[b, h, i])[0]:
                     c0, c1 = j * g.N, min((j + 1) * g.N, g.Lq)
                     rows.append(np.arange(c0, c1)[valid[c0:c1]])
-                keys = np.concatenate(rows)
+                keys = np.concatenate(rows) if rows else np.zeros(0, dtype=np.int64)
+                if keys.size == 0:
+                    O[b, h, r0:r1] = 0.0
+                    LSE[b, h, r0:r1] = -np.inf
+                    continue
                 s = (q[r0:r1] @ k[keys].T) * scale
                 m = s.max(axis=1, keepdims=True)
                 lse = m[:, 0] + np.log(np.exp(s - m).sum(axis=1))
@@ -292,7 +353,7 @@ def ssta_forward(d, q, k, v, q_text=None, k_text=None, v_text=None, q_tiles=None
     kp = tile_reorder(d, k, k_text)
     vp = tile_reorder(d, v, v_text)
     qbar, kbar = tile_pool(d, qp), tile_pool(d, kp)
-    S = tile_scores(d, qbar, kbar)
+    S = block_scores(d, qbar, kbar)
     sel = select_topk(d, S)
     kept = kept_mask(d, sel)
     idx, cnt = kept_lists(kept)

@@ -66,6 +66,11 @@ class Workload:
     seeds: tuple = (0,)
     note: str = ""
     extra: dict = field(default_factory=dict)
+    # mask modes (defaults: the headline configuration)
+    score_mode: str = "similarity"   # or "importance"
+    lam: float = 0.9                 # importance weight of the similarity term
+    combine: str = "union"           # or "and"
+    window_mode: str = "shift"       # or "truncate"
 
     @property
     def tokens(self) -> int:

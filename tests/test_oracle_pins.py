@@ -12,7 +12,15 @@
   the centred one) plus the pages' "within +-w/2" interior rule;
 * attention: torch's scaled_dot_product_attention in float64 on the raster
   tokens with a token-level mask built in raster space (dense, block-diagonal
-  and random kept sets), and torch.logsumexp for LSE.
+  and random kept sets), and torch.logsumexp for LSE; an empty kept set gives
+  O = 0 and LSE = -inf;
+* importance scores: closed forms (orthonormal keys: redundancy 1/2;
+  identical keys: redundancy 1), the independent identity
+  sum_{a != j} k_a . k_j = (sum_a k_a) . k_j - |k_j|^2, invariance to positive
+  scaling of the pooled vectors, lambda = 1 reducing to (cosine + 1) / 2, a
+  single tile and all-zero vectors; top-k on them by brute force;
+* truncated window: brute force over each axis and the pages' |c' - c| <= w/2
+  rule; AND combination: set intersection, and its two degenerate cases.
 
 Sources: "HunyuanVideo 1.5 Technical Report" (paper-graph-ui summary),
 section "SSTA: Selective and Sliding Tile Attention", Steps 1-4 and the
@@ -370,3 +378,147 @@ def test_flop_count_dense_case():
     kept = np.ones((1, w.H, g.NQ, g.NQ), dtype=bool)
     L = w.T * w.Y * w.X
     assert oracle.attention_flops(w, kept) == 4.0 * w.D * w.H * L * L
+
+
+# ---------------------------------------------------------------------------
+# Mask modes: importance scoring, truncated window, AND combination
+# ("Selective Mask Generation": Score_i = lambda Score_s - beta Score_r; the
+# blog's importance-sampling routine; Algorithm 1's M_sel AND M_sta; the
+# "within +-w/2" window rule)
+# ---------------------------------------------------------------------------
+
+def _imp_desc(lam=0.9, **kw):
+    return with_overrides(_desc(**kw), score_mode="importance", lam=lam)
+
+
+def test_importance_orthonormal_keys_closed_form():
+    # keys = distinct basis vectors, query i = basis vector i: cos = delta_ij, every key-key
+    # cosine off the diagonal is 0, so redundancy = (0 + 1) / 2 = 1/2 for every key
+    d = _imp_desc(lam=0.7)
+    NT, D = 5, 8
+    kb = np.eye(D)[None, None, :NT] * np.arange(1, NT + 1)[None, None, :, None]   # scaled: norm must not matter
+    qb = np.eye(D)[None, None, :NT] * 3.0
+    S = oracle.importance_scores(d, qb, kb)
+    want = 0.7 * (np.eye(NT) + 1.0) / 2.0 - 0.3 * 0.5
+    np.testing.assert_allclose(S[0, 0], want, atol=1e-15)
+
+
+def test_importance_identical_keys_have_full_redundancy():
+    d = _imp_desc(lam=0.6)
+    v = _rand((8,), 3)
+    kb = np.tile(v, (1, 1, 4, 1)) * np.array([1.0, 2.0, 0.5, 7.0])[None, None, :, None]
+    qb = _rand((1, 1, 3, 8), 4)
+    S = oracle.importance_scores(d, qb, kb)
+    cos = (qb[0, 0] @ v) / (np.linalg.norm(qb[0, 0], axis=1) * np.linalg.norm(v))
+    want = 0.6 * (cos[:, None] + 1.0) / 2.0 - 0.4 * 1.0
+    np.testing.assert_allclose(S[0, 0], np.broadcast_to(want, (3, 4)), atol=1e-14)
+
+
+def test_importance_matches_sum_vector_identity():
+    # independent route: sum_{a != j} k^_a . k^_j = (sum_a k^_a) . k^_j - |k^_j|^2
+    d = _imp_desc(lam=0.9)
+    qb, kb = _rand((2, 3, 7, 16), 5), _rand((2, 3, 9, 16), 6)
+    S = oracle.importance_scores(d, qb, kb)
+    qn = qb / np.linalg.norm(qb, axis=-1, keepdims=True)
+    kn = kb / np.linalg.norm(kb, axis=-1, keepdims=True)
+    u = kn.sum(axis=-2, keepdims=True)
+    dots = (kn * u).sum(-1) - (kn * kn).sum(-1)                  # [B,H,NT]
+    red = 0.5 + dots / (2.0 * (kb.shape[-2] - 1))
+    want = 0.9 * (np.einsum("bhid,bhjd->bhij", qn, kn) + 1.0) / 2.0 - 0.1 * red[..., None, :]
+    np.testing.assert_allclose(S, want, atol=1e-13)
+
+
+def test_importance_scale_invariance_and_lambda_one():
+    d = _imp_desc(lam=1.0)
+    qb, kb = _rand((1, 2, 6, 8), 7), _rand((1, 2, 6, 8), 8)
+    S = oracle.importance_scores(d, qb, kb)
+    S2 = oracle.importance_scores(d, qb * _rand((1, 2, 6, 1), 9) ** 2 + 0 * qb, kb * 5.0)
+    # positive per-row scales of q (squares of normals) and a global scale of k change nothing
+    np.testing.assert_allclose(S, S2, atol=1e-14)
+    cos = np.einsum("bhid,bhjd->bhij", qb / np.linalg.norm(qb, axis=-1, keepdims=True),
+                    kb / np.linalg.norm(kb, axis=-1, keepdims=True))
+    np.testing.assert_allclose(S, (cos + 1.0) / 2.0, atol=1e-14)   # lam = 1: similarity only
+
+
+def test_importance_single_tile_and_zero_vectors():
+    d = _imp_desc(lam=0.9)
+    S = oracle.importance_scores(d, _rand((1, 1, 1, 4), 1), _rand((1, 1, 1, 4), 2))
+    q = _rand((4,), 1); k = _rand((4,), 2)
+    cos = q @ k / (np.linalg.norm(q) * np.linalg.norm(k))
+    np.testing.assert_allclose(S[0, 0, 0, 0], 0.9 * (cos + 1) / 2, atol=1e-15)   # no other tile: no redundancy
+    qb = np.zeros((1, 1, 2, 4)); kb = np.zeros((1, 1, 3, 4))
+    S = oracle.importance_scores(d, qb, kb)                                     # zero vectors stay zero
+    np.testing.assert_allclose(S, 0.9 * 0.5 - 0.1 * 0.5, atol=1e-15)
+
+
+def test_importance_forward_selects_by_importance():
+    w = with_overrides(si.get_workload("tiny_f32"), score_mode="importance", topk=3)
+    x = si.make_inputs(w)
+    r = oracle.ssta_forward(w, *(None if x[k] is None else x[k].numpy()
+                                 for k in ("q", "k", "v", "q_text", "k_text", "v_text")))
+    S = oracle.importance_scores(w, r["qbar"], r["kbar"])
+    np.testing.assert_array_equal(r["scores"], S)
+    for h in range(w.H):
+        for i in range(oracle.geometry(w).NT):
+            assert set(np.nonzero(r["sel"][0, h, i])[0]) == _brute_topk(S[0, h, i].astype(np.float32), 3)
+
+
+def _brute_axis_window_truncated(n, w, c):
+    return {cc for cc in range(n) if c - w // 2 <= cc < c - w // 2 + w}
+
+
+@pytest.mark.parametrize("n", range(1, 8))
+@pytest.mark.parametrize("w", range(1, 10))
+def test_truncated_window_brute_force(n, w):
+    m = oracle.ssta_oracle._axis_window(n, w, truncate=True)
+    shift = oracle.ssta_oracle._axis_window(n, w)
+    for c in range(n):
+        got = set(np.nonzero(m[c])[0])
+        assert got == _brute_axis_window_truncated(n, w, c)
+        assert c in got
+        if w % 2 == 1:   # the pages' rule: |c' - c| <= w/2, cut at the grid
+            assert got == {cc for cc in range(n) if abs(cc - c) <= w // 2}
+        if c - w // 2 >= 0 and c - w // 2 + w <= n:   # away from the edges both modes agree
+            assert got == set(np.nonzero(shift[c])[0])
+
+
+def test_truncated_window_mask_is_product():
+    d = with_overrides(_desc(T=7, Y=9, X=10, tT=1, tY=2, tX=3, wT=3, wY=3, wX=5), window_mode="truncate")
+    g = oracle.geometry(d)
+    M = oracle.window_mask(d)
+    coords = [(a, b, c) for a in range(g.nT) for b in range(g.nY) for c in range(g.nX)]
+    for i, (a, b, c) in enumerate(coords):
+        want = np.array([a2 in _brute_axis_window_truncated(g.nT, 3, a) and b2 in _brute_axis_window_truncated(g.nY, 3, b)
+                         and c2 in _brute_axis_window_truncated(g.nX, 5, c) for (a2, b2, c2) in coords])
+        np.testing.assert_array_equal(M[i], want)
+
+
+def test_and_combination():
+    w = with_overrides(si.get_workload("tiny_f32"), combine="and", wT=1, wY=3, wX=3, topk=3, L_text=40)
+    g = oracle.geometry(w)
+    x = si.make_inputs(w)
+    r = oracle.ssta_forward(w, *(x[k].numpy() for k in ("q", "k", "v", "q_text", "k_text", "v_text")))
+    win = oracle.window_mask(w)
+    np.testing.assert_array_equal(r["kept"][:, :, : g.NT, : g.NT], r["sel"] & win[None, None])
+    assert np.all(r["kept"][:, :, : g.NT, g.NT:]) and np.all(r["kept"][:, :, g.NT:, :])
+    # top-k = all tiles: AND leaves the window; window = whole grid: AND leaves the selection
+    wa = with_overrides(w, topk=100)
+    ra = oracle.kept_mask(wa, oracle.select_topk(wa, r["scores"]))
+    np.testing.assert_array_equal(ra[:, :, : g.NT, : g.NT], np.broadcast_to(win, ra[:, :, : g.NT, : g.NT].shape))
+    wb = with_overrides(w, wT=9, wY=9, wX=9)
+    rb = oracle.kept_mask(wb, r["sel"])
+    np.testing.assert_array_equal(rb[:, :, : g.NT, : g.NT], r["sel"])
+
+
+def test_empty_kept_set_gives_zero_output():
+    # AND with a window that excludes every selected tile and no text: nothing to attend
+    w = with_overrides(si.get_workload("tiny_f32"), combine="and", wT=1, wY=1, wX=1, topk=1)
+    g = oracle.geometry(w)
+    x = si.make_inputs(w)
+    arrs = [x[k].numpy().astype(np.float64) for k in ("q", "k", "v")]
+    qp, kp, vp = (oracle.tile_reorder(w, a, None) for a in arrs)
+    kept = np.zeros((w.B, w.H, g.NQ, g.NQ), dtype=bool)
+    kept[:, :, 0, 1] = True                              # tile 0 keeps tile 1 only; the others keep nothing
+    O, L = oracle.attention(w, qp, kp, vp, kept)
+    assert np.all(O[:, :, g.N:] == 0.0) and np.all(np.isneginf(L[:, :, g.N:]))
+    assert np.all(np.isfinite(L[:, :, : g.N]))

@@ -34,6 +34,9 @@ lib = ctypes.CDLL(_LIB_PATH)
 
 SSTA_BF16 = 0
 SSTA_F32 = 1
+SCORE_MODES = {"similarity": 0, "importance": 1}
+COMBINE_MODES = {"union": 0, "and": 1}
+WINDOW_MODES = {"shift": 0, "truncate": 1}
 _STATUS = {0: "SSTA_OK", 1: "SSTA_ERR_INVALID_ARG", 2: "SSTA_ERR_UNSUPPORTED", 3: "SSTA_ERR_ALIGNMENT",
            4: "SSTA_ERR_WORKSPACE", 5: "SSTA_ERR_LAUNCH", 6: "SSTA_ERR_DEVICE_TIMEOUT",
            7: "SSTA_ERR_DEVICE_BOUNDS"}
@@ -43,7 +46,8 @@ class Desc(ctypes.Structure):
     """Mirror of ssta_desc."""
     _fields_ = [(n, ctypes.c_int) for n in
                 ("B", "H", "D", "T", "Y", "X", "tT", "tY", "tX", "wT", "wY", "wX", "topk", "L_text", "dtype")] + [
-        ("scale", ctypes.c_float)]
+        ("scale", ctypes.c_float), ("score_mode", ctypes.c_int), ("lambda_", ctypes.c_float),
+        ("combine", ctypes.c_int), ("window_mode", ctypes.c_int)]
 
 
 class _PlanInfo(ctypes.Structure):
@@ -93,7 +97,9 @@ def _check(code: int, where: str):
 def desc_from(w=None, **kw) -> Desc:
     """Build a descriptor from any object with the descriptor's field names (e.g. a
     workload), overridden by keyword arguments.  ``dtype`` may be "bf16"/"f32" or
-    the enum value."""
+    the enum value; the mask modes ``score_mode`` ("similarity"/"importance"),
+    ``combine`` ("union"/"and") and ``window_mode`` ("shift"/"truncate") may be
+    names or enum values, and ``lam`` is the importance weight (default 0.9)."""
     fields = {}
     for n in ("B", "H", "D", "T", "Y", "X", "tT", "tY", "tX", "wT", "wY", "wX", "topk", "L_text", "dtype"):
         if n in kw:
@@ -106,7 +112,14 @@ def desc_from(w=None, **kw) -> Desc:
     if isinstance(dt, str):
         fields["dtype"] = {"bf16": SSTA_BF16, "f32": SSTA_F32}[dt]
     scale = kw.get("scale", getattr(w, "scale", 0.0) if w is not None else 0.0) or 0.0
-    return Desc(**{k: int(v) for k, v in fields.items()}, scale=float(scale))
+
+    def mode(name, table, default):
+        v = kw.get(name, getattr(w, name, default) if w is not None else default)
+        return table[v] if isinstance(v, str) else int(v)
+    lam = float(kw.get("lam", getattr(w, "lam", 0.9) if w is not None else 0.9))
+    return Desc(**{k: int(v) for k, v in fields.items()}, scale=float(scale),
+                score_mode=mode("score_mode", SCORE_MODES, "similarity"), lambda_=lam,
+                combine=mode("combine", COMBINE_MODES, "union"), window_mode=mode("window_mode", WINDOW_MODES, "shift"))
 
 
 @dataclass

@@ -29,6 +29,10 @@ ssta_status make_geom(const ssta_desc* d, Geom* g) {
   if (d->topk < 0 || d->L_text < 0) return SSTA_ERR_INVALID_ARG;
   if (d->dtype != SSTA_BF16 && d->dtype != SSTA_F32) return SSTA_ERR_INVALID_ARG;
   if (!(d->scale >= 0.0f) || isinf(d->scale)) return SSTA_ERR_INVALID_ARG;
+  if (d->score_mode != SSTA_SCORE_SIMILARITY && d->score_mode != SSTA_SCORE_IMPORTANCE) return SSTA_ERR_INVALID_ARG;
+  if (d->score_mode == SSTA_SCORE_IMPORTANCE && !(d->lambda >= 0.0f && d->lambda <= 1.0f)) return SSTA_ERR_INVALID_ARG;
+  if (d->combine != SSTA_COMBINE_UNION && d->combine != SSTA_COMBINE_AND) return SSTA_ERR_INVALID_ARG;
+  if (d->window_mode != SSTA_WINDOW_SHIFT && d->window_mode != SSTA_WINDOW_TRUNCATE) return SSTA_ERR_INVALID_ARG;
   if ((int64_t)d->B * d->H > 65535) return SSTA_ERR_UNSUPPORTED;
   if (d->D != 128) return SSTA_ERR_UNSUPPORTED;
   const int64_t N = (int64_t)d->tT * d->tY * d->tX;
@@ -62,6 +66,11 @@ ssta_status make_geom(const ssta_desc* d, Geom* g) {
   x.dtype = d->dtype;
   x.esize = d->dtype == SSTA_BF16 ? 2 : 4;
   x.scale = d->scale > 0.0f ? d->scale : 1.0f / sqrtf((float)d->D);
+  x.score_mode = d->score_mode;
+  x.lambda = d->score_mode == SSTA_SCORE_IMPORTANCE ? d->lambda : 0.0f;
+  x.combine = d->combine;
+  x.window_mode = d->window_mode;
+  x.norm_blocks = ceil_div(x.NT, 128);
   *g = x;
   return SSTA_OK;
 }
@@ -135,9 +144,15 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
   float* qbar = reinterpret_cast<float*>(w + ws.qbar);
   float* kbar = reinterpret_cast<float*>(w + ws.kbar);
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(w + ws.scores);
+  const bool imp = g.score_mode == SSTA_SCORE_IMPORTANCE;
+  const ImportanceBufs ib = imp ? ImportanceBufs{reinterpret_cast<float*>(w + ws.inv_nq), reinterpret_cast<float*>(w + ws.inv_nk),
+                                                 reinterpret_cast<float*>(w + ws.ksum), reinterpret_cast<float*>(w + ws.red)}
+                                : ImportanceBufs{nullptr, nullptr, nullptr, nullptr};
   // the pool kernel also clears the status word
   cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(w + ws.status), s);
-  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, scores, s);
+  if (e == cudaSuccess && imp) e = launch_tile_norms(g, qbar, kbar, ib, s);
+  if (e == cudaSuccess && imp) e = launch_tile_redundancy(g, kbar, ib, s);
+  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return from_cuda(e);
 }

@@ -28,6 +28,11 @@ struct Geom {
   int esize;            // bytes per element (2 or 4)
   int dtype;
   float scale;          // softmax scale
+  int score_mode;       // ssta_score_mode
+  float lambda;         // importance score weight
+  int combine;          // ssta_combine
+  int window_mode;      // ssta_window
+  int norm_blocks;      // 128-tile blocks of the importance pre-pass = ceil(NT/128)
 };
 
 // Workspace layout of ssta_build_block_mask (byte offsets, 256-aligned).
@@ -35,11 +40,24 @@ struct MaskWorkspace {
   size_t status;   // int32 device status word
   size_t qbar;     // fp32 [BH, D, NT] (channel-major)
   size_t kbar;     // fp32 [BH, D, NT] (channel-major)
-  size_t scores;   // fp32 [BH, NT, NT]
+  size_t inv_nq;   // importance score only: fp32 [BH, NT], 1 / |Qbar_i| (0 for a zero mean)
+  size_t inv_nk;   //   fp32 [BH, NT], 1 / |Kbar_j|
+  size_t ksum;     //   fp32 [BH, norm_blocks, D], per 128-tile block sum of unit Kbar_j
+  size_t red;      //   fp32 [BH, NT], redundancy of key tile j
+  size_t scores;   // fp32 [BH, NT, NT]; absent when `with_scores` is false
   size_t total;
 };
 
-MaskWorkspace mask_workspace_layout(const Geom& g);
+// Offsets from 0; `with_scores` = false when the caller supplies the score matrix.
+MaskWorkspace mask_workspace_layout(const Geom& g, bool with_scores = true);
+
+// The importance buffers of a mask workspace at `base` (all NULL for the similarity score).
+struct ImportanceBufs {
+  float* inv_nq;
+  float* inv_nk;
+  float* ksum;
+  float* red;
+};
 
 // Validate a descriptor and derive every size (host only, no CUDA call).
 ssta_status make_geom(const ssta_desc* d, Geom* g);
@@ -53,8 +71,14 @@ cudaError_t launch_tile_unorder(const Geom& g, const void* packed, void* raster,
 // finished, so a mask build needs no separate reset of its status word.
 cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, float* qbar, float* kbar,
                              int32_t* status, cudaStream_t s);
-cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
-                               cudaStream_t s);
+// Importance score only: per-tile inverse norms and per-block sums of unit key means,
+// then the per-key redundancy.  Both wait for the previous kernel (programmatic launch).
+cudaError_t launch_tile_norms(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
+                              cudaStream_t s);
+cudaError_t launch_tile_redundancy(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s);
+// Block scores: raw dot products, or the importance score when ib.red != NULL.
+cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
+                               float* scores, cudaStream_t s);
 cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
                                    cudaStream_t s);
 cudaError_t launch_attention_f32(const Geom& g, const float* qp, const float* kp, const float* vp,

@@ -11,15 +11,20 @@
 //                         valid q and k rows with 16-byte coalesced loads and
 //                         reduces per-channel fp32 sums across row groups; the
 //                         means are stored channel-major for the score kernel.
+//   tile_norms_kernel,    importance score only: inverse norms of the tile
+//   tile_redundancy_kernel means and the per-key redundancy (mean key-key
+//                         similarity to the other key tiles), O(NT*D) per head
+//                         through the sum of the unit key means.
 //   tile_scores_kernel    fp32 SIMT, 128x128 score blocks per CTA, 8x8 per
 //                         thread, 16-channel stages double-buffered in shared
 //                         memory by cp.async, channels summed in order 0..D-1
-//                         with FMA (packed f32x2, two columns per instruction).
+//                         with FMA (packed f32x2, two columns per instruction);
+//                         the importance transform is applied in the epilogue.
 //   select_and_list_kernel one warp per (head, query tile): top-k over scores
 //                         held in registers as order-preserving 32-bit keys
 //                         (bitwise binary search for the k-th key with warp-wide
 //                         counts, ties to the lower tile index by ballots in
-//                         index order), OR-ed word by word with the window
+//                         index order), OR-ed (or AND-ed) word by word with the window
 //                         (contiguous index ranges) and compacted into the
 //                         ascending kept list by a warp prefix sum.
 #include "ssta_internal.h"
@@ -144,6 +149,75 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
   }
 }
 
+// Step 2, importance score, pre-pass 1 (one CTA per 128 tiles of one head, one
+// thread per tile): the inverse L2 norm of each tile mean of q and of k (0 for an
+// all-zero mean), and this block's sum of the unit-length key means, one value per
+// channel, reduced in a fixed order (warp shuffle tree, then the four warps in
+// order) so the result does not depend on scheduling.
+__global__ void __launch_bounds__(128)
+tile_norms_kernel(Geom g, const float* __restrict__ qbar_t, const float* __restrict__ kbar_t, ImportanceBufs ib) {
+  allow_dependents();
+  grid_dependency_wait();   // the pooled means are written by the previous kernel
+  __shared__ float part[4][128];
+  const int64_t bh = blockIdx.y;
+  const int NT = g.NT, D = g.D;
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  const bool valid = c < NT;
+  const float* qh = qbar_t + bh * D * (int64_t)NT;
+  const float* kh = kbar_t + bh * D * (int64_t)NT;
+  float sq = 0.f, sk = 0.f;
+  if (valid) {
+    for (int d = 0; d < D; ++d) {
+      const float a = qh[(int64_t)d * NT + c], b = kh[(int64_t)d * NT + c];
+      sq = fmaf(a, a, sq);
+      sk = fmaf(b, b, sk);
+    }
+  }
+  const float iq = sq > 0.f ? 1.0f / sqrtf(sq) : 0.f;
+  const float ik = sk > 0.f ? 1.0f / sqrtf(sk) : 0.f;
+  if (valid) {
+    ib.inv_nq[bh * NT + c] = iq;
+    ib.inv_nk[bh * NT + c] = ik;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int d = 0; d < D; ++d) {
+    float v = valid ? kh[(int64_t)d * NT + c] * ik : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+    if (lane == 0) part[warp][d] = v;
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += 128)
+    ib.ksum[(bh * g.norm_blocks + blockIdx.x) * D + d] = ((part[0][d] + part[1][d]) + part[2][d]) + part[3][d];
+}
+
+// Step 2, importance score, pre-pass 2 (same grid): the redundancy of key tile j,
+// the mean over the other key tiles j' of (u_j' . u_j + 1) / 2 with u the unit key
+// means, through sum_{j' != j} u_j' . u_j = (sum_j' u_j') . u_j - |u_j|^2; the
+// per-block sums are added in block order.  0 when the grid has one tile.
+__global__ void __launch_bounds__(128)
+tile_redundancy_kernel(Geom g, const float* __restrict__ kbar_t, ImportanceBufs ib) {
+  allow_dependents();
+  grid_dependency_wait();   // the per-block key sums are written by the previous kernel
+  __shared__ float usum[128];
+  const int64_t bh = blockIdx.y;
+  const int NT = g.NT, D = g.D;
+  for (int d = threadIdx.x; d < D; d += 128) {
+    float a = 0.f;
+    for (int b = 0; b < g.norm_blocks; ++b) a += ib.ksum[(bh * g.norm_blocks + b) * D + d];
+    usum[d] = a;
+  }
+  __syncthreads();
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  if (c >= NT) return;
+  const float* kh = kbar_t + bh * D * (int64_t)NT;
+  float dot = 0.f;
+  for (int d = 0; d < D; ++d) dot = fmaf(kh[(int64_t)d * NT + c], usum[d], dot);
+  const float ik = ib.inv_nk[bh * NT + c];
+  const float self = ik > 0.f ? 1.0f : 0.f;             // |u_j|^2
+  ib.red[bh * NT + c] = NT > 1 ? 0.5f + (dot * ik - self) / (2.0f * (float)(NT - 1)) : 0.f;
+}
+
 // Step 2, Score_s = Qbar Kbar^T.  One CTA computes a 128 x 128 block of scores
 // of one head with 256 threads; thread (ty, tx) of a 16 x 16 grid owns rows
 // {4ty..4ty+3, 64+4ty..64+4ty+3} and the same pattern of columns, i.e. 8 x 8
@@ -212,7 +286,7 @@ __device__ __forceinline__ void score_stage_copy(float (*qs)[kScoreBlock], float
 template <bool kVec>
 __global__ void __launch_bounds__(256, 2)
 tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __restrict__ kbar_t,
-                   float* __restrict__ scores) {
+                   ImportanceBufs ib, float* __restrict__ scores) {
   __shared__ __align__(16) float qs[2][kScoreStage][kScoreBlock];
   __shared__ __align__(16) float ks[2][kScoreStage][kScoreBlock];
   const int64_t bh = blockIdx.z;
@@ -261,17 +335,34 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
     __syncthreads();   // every thread is done with buffer buf before it is refilled
   }
   float* sh = scores + bh * NT * (int64_t)NT;
+  // importance score: lambda (cos + 1) / 2 - (1 - lambda) red_j, cos = dot / (|Qbar_i| |Kbar_j|)
+  const bool imp = ib.red != nullptr;
+  float ck[8], rk[8];
+  if (imp) {
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int j = j0 + (b < 4 ? 4 * tx + b : 64 + 4 * tx + b - 4);
+      ck[b] = j < NT ? ib.inv_nk[bh * NT + j] : 0.f;
+      rk[b] = j < NT ? (1.0f - g.lambda) * ib.red[bh * NT + j] : 0.f;
+    }
+  }
 #pragma unroll
   for (int a = 0; a < 8; ++a) {
     const int i = i0 + (a < 4 ? 4 * ty + a : 64 + 4 * ty + a - 4);
     if (i >= NT) continue;
     float* srow = sh + (int64_t)i * NT;
+    const float cq = imp ? ib.inv_nq[bh * NT + i] : 0.f;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int j = j0 + 64 * half + 4 * tx;
       float v[4];
       f2_unpack(acc[a][2 * half], v[0], v[1]);
       f2_unpack(acc[a][2 * half + 1], v[2], v[3]);
+      if (imp) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          v[b] = g.lambda * 0.5f * (v[b] * cq * ck[4 * half + b] + 1.0f) - rk[4 * half + b];
+      }
       if constexpr (kVec) {
         if (j < NT) *reinterpret_cast<float4*>(srow + j) = make_float4(v[0], v[1], v[2], v[3]);
       } else {
@@ -313,8 +404,9 @@ __device__ __forceinline__ uint32_t range_bits(int word, int lo, int hi) {
 //    warp-wide counts (upper 16 bits over all keys, lower 16 bits over the keys
 //    sharing that upper half); keys above it are taken, and keys equal to it are
 //    taken in ascending tile order until k are chosen (ties to the lower index);
-//  * the window (Step 3) as unions of contiguous index ranges, one per (t, y)
-//    tile row of the window, OR-ed word by word with the selection;
+//  * the window (Step 3, shifted or truncated at the grid edges) as unions of
+//    contiguous index ranges, one per (t, y) tile row of the window, OR-ed (union)
+//    or AND-ed (Algorithm 1's intersection) word by word with the selection;
 //  * the union (Step 4) written as an ascending list by a warp prefix sum over the
 //    32-tile words, followed by the text tiles and -1 padding.
 // Text query tiles keep every tile.
@@ -436,9 +528,17 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
     }
     // ---- window rows: for each (t, y) tile row of the window, a contiguous x range
     const int cX = i % g.nX, cY = (i / g.nX) % g.nY, cT = i / (g.nX * g.nY);
-    const int sT = window_start(cT, g.wT, g.nT), sY = window_start(cY, g.wY, g.nY),
-              sX = window_start(cX, g.wX, g.nX);
-    const int eT = sT + min(g.wT, g.nT), eY = sY + min(g.wY, g.nY), nwX = min(g.wX, g.nX);
+    int sT, sY, sX, eT, eY, nwX;
+    if (g.window_mode == SSTA_WINDOW_TRUNCATE) {
+      // [c - w/2, c - w/2 + w) cut at the grid
+      const int lT = cT - g.wT / 2, lY = cY - g.wY / 2, lX = cX - g.wX / 2;
+      sT = max(lT, 0); eT = min(lT + g.wT, g.nT);
+      sY = max(lY, 0); eY = min(lY + g.wY, g.nY);
+      sX = max(lX, 0); nwX = min(lX + g.wX, g.nX) - sX;
+    } else {
+      sT = window_start(cT, g.wT, g.nT); sY = window_start(cY, g.wY, g.nY); sX = window_start(cX, g.wX, g.nX);
+      eT = sT + min(g.wT, g.nT); eY = sY + min(g.wY, g.nY); nwX = min(g.wX, g.nX);
+    }
 #pragma unroll
     for (int q = 0; q < (SLOTS + 31) / 32; ++q) {
       const int word = lane + 32 * q;
@@ -449,7 +549,7 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
           const int lo = (wt * g.nY + wy) * g.nX + sX;
           win |= range_bits(word, lo, lo + nwX);
         }
-      myword[q] |= win;
+      myword[q] = g.combine == SSTA_COMBINE_AND ? (myword[q] & win) : (myword[q] | win);
     }
     // ---- compaction: exclusive prefix of the kept counts over words in ascending order
 #pragma unroll
@@ -486,15 +586,23 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
 
 }  // namespace
 
-MaskWorkspace mask_workspace_layout(const Geom& g) {
+MaskWorkspace mask_workspace_layout(const Geom& g, bool with_scores) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t bh = (size_t)g.B * g.H;
-  MaskWorkspace w;
+  MaskWorkspace w{};
   w.status = 0;
   w.qbar = 256;
   w.kbar = w.qbar + up(bh * g.NT * g.D * sizeof(float));
-  w.scores = w.kbar + up(bh * g.NT * g.D * sizeof(float));
-  w.total = w.scores + up(bh * g.NT * (size_t)g.NT * sizeof(float));
+  size_t end = w.kbar + up(bh * g.NT * g.D * sizeof(float));
+  if (g.score_mode == SSTA_SCORE_IMPORTANCE) {
+    w.inv_nq = end;
+    w.inv_nk = w.inv_nq + up(bh * g.NT * sizeof(float));
+    w.ksum = w.inv_nk + up(bh * g.NT * sizeof(float));
+    w.red = w.ksum + up(bh * g.norm_blocks * g.D * sizeof(float));
+    end = w.red + up(bh * g.NT * sizeof(float));
+  }
+  w.scores = end;
+  w.total = end + (with_scores ? up(bh * g.NT * (size_t)g.NT * sizeof(float)) : 0);
   return w;
 }
 
@@ -514,13 +622,24 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
                           status);
 }
 
-cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, float* scores,
-                               cudaStream_t s) {
+cudaError_t launch_tile_norms(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
+                              cudaStream_t s) {
+  if ((int64_t)g.B * g.H == 0) return cudaSuccess;
+  return launch_dependent(tile_norms_kernel, dim3(g.norm_blocks, g.B * g.H), dim3(128), 0, s, g, qbar, kbar, ib);
+}
+
+cudaError_t launch_tile_redundancy(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s) {
+  if ((int64_t)g.B * g.H == 0) return cudaSuccess;
+  return launch_dependent(tile_redundancy_kernel, dim3(g.norm_blocks, g.B * g.H), dim3(128), 0, s, g, kbar, ib);
+}
+
+cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
+                               float* scores, cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
   dim3 grid(ceil_div(g.NT, kScoreBlock), ceil_div(g.NT, kScoreBlock), g.B * g.H);
   if (g.NT % 4 == 0)
-    return launch_dependent(tile_scores_kernel<true>, grid, dim3(256), 0, s, g, qbar, kbar, scores);
-  return launch_dependent(tile_scores_kernel<false>, grid, dim3(256), 0, s, g, qbar, kbar, scores);
+    return launch_dependent(tile_scores_kernel<true>, grid, dim3(256), 0, s, g, qbar, kbar, ib, scores);
+  return launch_dependent(tile_scores_kernel<false>, grid, dim3(256), 0, s, g, qbar, kbar, ib, scores);
 }
 
 cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,

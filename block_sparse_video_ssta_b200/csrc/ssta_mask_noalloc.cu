@@ -49,7 +49,6 @@ ssta_status scratch_address(void** out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) % 16) == 0; }
-size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 }  // namespace ssta
@@ -62,14 +61,11 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
-  // scratch layout: status word | qbar | kbar | scores (only without tile_scores)
+  // scratch layout: the workspace layout of ssta_build_block_mask, without the score
+  // matrix when the caller supplies it
   const size_t bh = (size_t)g.B * g.H;
-  const size_t off_qbar = 256;
-  const size_t off_kbar = off_qbar + up256(bh * g.NT * g.D * sizeof(float));
-  const size_t off_scores = off_kbar + up256(bh * g.NT * g.D * sizeof(float));
-  const size_t scores_bytes = tile_scores != nullptr ? 0 : up256(bh * g.NT * (size_t)g.NT * sizeof(float));
-  const size_t total = off_scores + scores_bytes;
-  if (total > (size_t)SSTA_STATIC_SCRATCH_BYTES) return SSTA_ERR_WORKSPACE;
+  const MaskWorkspace ws = mask_workspace_layout(g, tile_scores == nullptr);
+  if (ws.total > (size_t)SSTA_STATIC_SCRATCH_BYTES) return SSTA_ERR_WORKSPACE;
   const bool empty = bh == 0;
   if (!empty && (q_packed == nullptr || k_packed == nullptr || kv_idx == nullptr || kv_cnt == nullptr))
     return SSTA_ERR_INVALID_ARG;
@@ -82,12 +78,18 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   uint8_t* base = static_cast<uint8_t*>(base_v);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (empty) return cudaMemsetAsync(base, 0, sizeof(int32_t), s) == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;
-  float* qbar = reinterpret_cast<float*>(base + off_qbar);
-  float* kbar = reinterpret_cast<float*>(base + off_kbar);
-  float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(base + off_scores);
+  float* qbar = reinterpret_cast<float*>(base + ws.qbar);
+  float* kbar = reinterpret_cast<float*>(base + ws.kbar);
+  float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(base + ws.scores);
+  const bool imp = g.score_mode == SSTA_SCORE_IMPORTANCE;
+  const ImportanceBufs ib = imp ? ImportanceBufs{reinterpret_cast<float*>(base + ws.inv_nq), reinterpret_cast<float*>(base + ws.inv_nk),
+                                                 reinterpret_cast<float*>(base + ws.ksum), reinterpret_cast<float*>(base + ws.red)}
+                                : ImportanceBufs{nullptr, nullptr, nullptr, nullptr};
   // the pool kernel also clears the status word
-  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(base), s);
-  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, scores, s);
+  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(base + ws.status), s);
+  if (e == cudaSuccess && imp) e = launch_tile_norms(g, qbar, kbar, ib, s);
+  if (e == cudaSuccess && imp) e = launch_tile_redundancy(g, kbar, ib, s);
+  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;
 }

@@ -69,7 +69,31 @@ typedef enum {
 
 typedef enum { SSTA_BF16 = 0, SSTA_F32 = 1 } ssta_dtype;
 
-/* Problem descriptor.  All fields are plain integers; see the layouts above. */
+/* Block score ranked by top-k (Step 2, "Selective Mask Generation"). */
+typedef enum {
+  SSTA_SCORE_SIMILARITY = 0, /* Score_s = Qbar . Kbar (raw dot product of the tile means) */
+  SSTA_SCORE_IMPORTANCE = 1  /* lambda (cos(Qbar, Kbar) + 1) / 2 - (1 - lambda) * redundancy, where the
+                                redundancy of key tile j is the mean over the other key tiles j' of
+                                (cos(Kbar_j', Kbar_j) + 1) / 2 (0 when NT = 1); an all-zero mean has
+                                cosine 0 with everything */
+} ssta_score_mode;
+
+/* How selection and window combine (Step 4). */
+typedef enum {
+  SSTA_COMBINE_UNION = 0,    /* selected OR in the window */
+  SSTA_COMBINE_AND = 1       /* selected AND in the window (Algorithm 1 as printed) */
+} ssta_combine;
+
+/* Window at the grid edges (Step 3).  The window of tile c on an axis of n tiles
+ * covers [c - w/2, c - w/2 + w) (integer w/2). */
+typedef enum {
+  SSTA_WINDOW_SHIFT = 0,     /* slid inward so it keeps min(w, n) tiles */
+  SSTA_WINDOW_TRUNCATE = 1   /* cut at 0 and n */
+} ssta_window;
+
+/* Problem descriptor.  All fields are plain integers or floats; see the layouts
+ * above.  A descriptor whose mode fields are all zero selects the similarity
+ * score, the union and the shifted window. */
 typedef struct {
   int B, H, D;      /* batch, heads, head dim (D must be 128) */
   int T, Y, X;      /* valid latent grid: frames, height, width (each >= 1) */
@@ -79,6 +103,11 @@ typedef struct {
   int L_text;       /* appended text tokens (>= 0) */
   int dtype;        /* ssta_dtype */
   float scale;      /* softmax scale; 0 means 1/sqrt(D) */
+  int score_mode;   /* ssta_score_mode */
+  float lambda;     /* importance score: weight of the similarity term, in [0, 1] (the pages use 0.9);
+                       ignored by the similarity score */
+  int combine;      /* ssta_combine */
+  int window_mode;  /* ssta_window */
 } ssta_desc;
 
 /* Sizes derived from a descriptor. */
@@ -99,7 +128,10 @@ typedef struct {
  * ssta_plan — derive every size from `desc` (host only, no CUDA call).
  * Step 1, "3D Block Partition": NT = ceil(T/tT)*ceil(Y/tY)*ceil(X/tX).
  * max_kept = NT + num_text_tiles when L_text > 0 (text query tiles attend every
- * tile), else min(NT, topk + window_tiles).
+ * tile), else min(NT, topk + window_tiles).  window_tiles is the largest window
+ * (with SSTA_WINDOW_TRUNCATE edge tiles keep fewer).  workspace_bytes depends on
+ * score_mode (the importance score keeps per-tile norms and redundancies).
+ * Returns SSTA_ERR_INVALID_ARG also for an unknown mode or lambda outside [0, 1].
  * Returns SSTA_ERR_INVALID_ARG for malformed descriptors, SSTA_ERR_UNSUPPORTED
  * when D != 128, N > 4096, NT > 2048, B*H > 65535 or Lq >= 2^31.
  */
@@ -117,15 +149,18 @@ ssta_status ssta_tile_reorder(const ssta_desc* desc, const void* x_raster, const
 
 /*
  * ssta_build_block_mask — Steps 2-4 up to the mask: per (b, h, video tile) mean
- * of q and k over the tile's valid tokens; fp32 scores S = Qbar Kbar^T
- * (Step 2, Score_s); per query tile the top-k key tiles by score, ties to the
- * lower tile index (Step 2, Topk/Indexes2mask); union with the sliding tile
- * window, which slides inward at the grid edges so it always spans
- * min(w, n) tiles per axis (Step 3), and with every text tile; text query tiles
- * keep every tile (Step 4, union reading).  Writes the compact lists.
+ * of q and k over the tile's valid tokens; fp32 block scores (Step 2: Score_s =
+ * Qbar Kbar^T, or the importance score of desc->score_mode); per query tile the
+ * top-k key tiles by score, ties to the lower tile index (Step 2,
+ * Topk/Indexes2mask); combined (desc->combine: union, or AND) with the sliding
+ * tile window (Step 3; desc->window_mode: slid inward at the grid edges so it
+ * always spans min(w, n) tiles per axis, or truncated), and with every text tile;
+ * text query tiles keep every tile (Step 4).  Writes the compact lists; a video
+ * query tile can keep no tile at all (AND, no text), its count is then 0.
  *   q_packed, k_packed [B,H,Lq,D] (read; pad rows are ignored),
  *   kv_idx [B,H,NQ,max_kept] and kv_cnt [B,H,NQ] (written),
- *   tile_scores [B,H,NT,NT] fp32 (written when non-NULL, else kept in workspace),
+ *   tile_scores [B,H,NT,NT] fp32: the block scores top-k ranks (written when
+ *   non-NULL, else kept in workspace),
  *   workspace >= info.workspace_bytes (contents overwritten).
  */
 ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, const void* k_packed,
@@ -137,6 +172,7 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
  * row, softmax(q k^T * scale) v over the valid keys of the kept key tiles of
  * its query tile (full attention inside each kept tile; key tiles that are not
  * listed are never read).  Pad query rows are computed but carry no meaning.
+ * A query tile with no valid kept key gets O = 0 and LSE = -inf.
  *   q/k/v_packed [B,H,Lq,D] (read), kv_idx/kv_cnt as written by
  *   ssta_build_block_mask (read; ids must be < NQ and ascending order is not
  *   required), o_packed [B,H,Lq,D] (written, dtype), lse [B,H,Lq] fp32

@@ -18,9 +18,9 @@ P = ctypes.c_void_p
 
 def desc(**kw):
     base = dict(B=1, H=2, D=128, T=4, Y=8, X=8, tT=2, tY=4, tX=4, wT=1, wY=1, wX=1, topk=2, L_text=0,
-                dtype=S.SSTA_F32)
+                dtype=S.SSTA_F32, scale=0.0)
     base.update(kw)
-    return S.Desc(**base, scale=0.0)
+    return S.Desc(**base)
 
 
 def call(name, *args):
@@ -36,6 +36,19 @@ for field, val, _ in [("B", -1, 1), ("T", 0, 1), ("tX", 0, 1), ("wY", 0, 1), ("t
                       ("L_text", -2, 1), ("dtype", 7, 1)]:
     cases.append((f"plan_bad_{field}", call("ssta_plan", ctypes.byref(desc(**{field: val})), ctypes.byref(info))))
 cases.append(("plan_D64", call("ssta_plan", ctypes.byref(desc(D=64)), ctypes.byref(info))))
+for name, kw in [("score_mode", dict(score_mode=2)), ("lambda_high", dict(score_mode=1, lambda_=1.5)),
+                 ("lambda_nan", dict(score_mode=1, lambda_=float("nan"))), ("combine", dict(combine=3)),
+                 ("window_mode", dict(window_mode=-1))]:
+    cases.append((f"plan_bad_{name}", call("ssta_plan", ctypes.byref(desc(**kw)), ctypes.byref(info))))
+# lambda is ignored by the similarity score; modes in range are accepted
+cases.append(("plan_similarity_ignores_lambda", call("ssta_plan", ctypes.byref(desc(lambda_=float("nan"))),
+                                                     ctypes.byref(info))))
+cases.append(("plan_all_modes", call("ssta_plan", ctypes.byref(desc(score_mode=1, lambda_=0.9, combine=1,
+                                                                    window_mode=1)), ctypes.byref(info))))
+_sim = S._PlanInfo(); _imp = S._PlanInfo()
+call("ssta_plan", ctypes.byref(desc()), ctypes.byref(_sim))
+call("ssta_plan", ctypes.byref(desc(score_mode=1, lambda_=0.9)), ctypes.byref(_imp))
+cases.append(("plan_importance_workspace_larger", 0 if _imp.workspace_bytes > _sim.workspace_bytes else 99))
 cases.append(("plan_tile_too_big", call("ssta_plan", ctypes.byref(desc(tT=16, tY=16, tX=32)), ctypes.byref(info))))
 cases.append(("plan_too_many_tiles", call("ssta_plan", ctypes.byref(desc(T=64, Y=64, X=64, tT=1, tY=1, tX=1)),
                                          ctypes.byref(info))))

@@ -50,7 +50,7 @@ def run_gpu(w, inputs, want_scores=True):
 def oracle_mask(w, q_np, k_np, qt_np, kt_np):
     qp = oracle.tile_reorder(w, q_np, qt_np)
     kp = oracle.tile_reorder(w, k_np, kt_np)
-    S64 = oracle.tile_scores(w, oracle.tile_pool(w, qp), oracle.tile_pool(w, kp))
+    S64 = oracle.block_scores(w, oracle.tile_pool(w, qp), oracle.tile_pool(w, kp))
     sel = oracle.select_topk(w, S64)
     kept = oracle.kept_mask(w, sel)
     return qp, kp, S64, kept
@@ -97,7 +97,8 @@ def compare_masks(w, kept_gpu, kept_ref, S64):
 
 
 def compare_attention(w, O_gpu, lse_gpu, O_ref, lse_ref, rows_mask):
-    """Compare on packed rows selected by rows_mask [B,H,Lq] (valid rows of agreeing tiles)."""
+    """Compare on packed rows selected by rows_mask [B,H,Lq] (valid rows of agreeing tiles).
+    A row that keeps no key must be O = 0, LSE = -inf on both sides."""
     tol = TOL[w.dtype]
     a = O_gpu[rows_mask]
     b = O_ref[rows_mask]
@@ -105,7 +106,9 @@ def compare_attention(w, O_gpu, lse_gpu, O_ref, lse_ref, rows_mask):
     err = np.abs(a - b)
     max_abs = float(err.max()) if err.size else 0.0
     rel = float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
-    lse_err = float(np.abs(lse_gpu[rows_mask] - lse_ref[rows_mask]).max()) if err.size else 0.0
+    la, lb = lse_gpu[rows_mask], lse_ref[rows_mask]
+    empty = np.isneginf(la) & np.isneginf(lb)                 # rows with no kept key on both sides
+    lse_err = float(np.where(empty, 0.0, np.abs(la - lb)).max()) if err.size else 0.0
     assert max_abs <= tol["o_max"], f"O max-abs {max_abs} > {tol['o_max']}"
     assert rel <= tol["o_rel"], f"O rel-L2 {rel} > {tol['o_rel']}"
     assert lse_err <= tol["lse_max"], f"LSE max-abs {lse_err} > {tol['lse_max']}"

@@ -60,11 +60,14 @@ def test_host_validation_codes():
     assert r.returncode == 0, r.stderr
     got = dict(line.split() for line in r.stdout.strip().splitlines())
     got = {k: int(v) for k, v in got.items()}
-    INVALID, UNSUP, ALIGN, WS = 1, 2, 3, 4
+    OK, INVALID, UNSUP, ALIGN, WS = 0, 1, 2, 3, 4
     expect = {
         "plan_null_desc": INVALID, "plan_null_info": INVALID, "plan_bad_B": INVALID, "plan_bad_T": INVALID,
         "plan_bad_tX": INVALID, "plan_bad_wY": INVALID, "plan_bad_topk": INVALID, "plan_bad_L_text": INVALID,
-        "plan_bad_dtype": INVALID, "plan_D64": UNSUP, "plan_tile_too_big": UNSUP, "plan_too_many_tiles": UNSUP,
+        "plan_bad_dtype": INVALID, "plan_bad_score_mode": INVALID, "plan_bad_lambda_high": INVALID,
+        "plan_bad_lambda_nan": INVALID, "plan_bad_combine": INVALID, "plan_bad_window_mode": INVALID,
+        "plan_similarity_ignores_lambda": OK, "plan_all_modes": OK, "plan_importance_workspace_larger": OK,
+        "plan_D64": UNSUP, "plan_tile_too_big": UNSUP, "plan_too_many_tiles": UNSUP,
         "plan_neg_scale": INVALID, "reorder_null_out": INVALID, "reorder_misaligned": ALIGN,
         "reorder_text_missing": INVALID, "unorder_null_in": INVALID, "unorder_misaligned_text": ALIGN,
         "mask_no_workspace": WS, "mask_small_workspace": WS, "mask_ws_misaligned": ALIGN, "mask_null_q": INVALID,

@@ -26,10 +26,12 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("name,with_scores", [("tiny_f32", True), ("small_bf16", False),
-                                              ("small_bf16", True), ("p720_5s_bf16", False)])
-def test_noalloc_matches_workspace_entry_point(cuda_ok, name, with_scores):
-    w = si.get_workload(name)
+@pytest.mark.parametrize("name,with_scores,mode", [("tiny_f32", True, "similarity"), ("small_bf16", False, "similarity"),
+                                                   ("small_bf16", True, "similarity"),
+                                                   ("p720_5s_bf16", False, "similarity"),
+                                                   ("small_bf16", False, "importance")])
+def test_noalloc_matches_workspace_entry_point(cuda_ok, name, with_scores, mode):
+    w = si.with_overrides(si.get_workload(name), score_mode=mode)
     x = si.make_inputs(w, 2, device="cuda")
     d = S.desc_from(w)
     p = S.ssta_plan(d)

@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 METRIC = "SSTA fwd ms/call & effective TFLOPS (kept blocks) at 720p-10s latent; % bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 LAUNCHES_PER_STEP = 8   # 3 reorder + pool + scores + select-and-list + attention + unorder
+                        # (+ norms and redundancy with the importance score)
 
 
 def load_peaks():
@@ -178,7 +179,7 @@ def oracle_sample(w, x_cpu, heads=(0,), tile_stride=64, max_seconds=None):
     q, k, v = (conv(x_cpu[n]) for n in ("q", "k", "v"))
     qt, kt, vt = (conv(x_cpu[n]) for n in ("q_text", "k_text", "v_text"))
     qp, kp, vp = oracle.tile_reorder(w, q, qt), oracle.tile_reorder(w, k, kt), oracle.tile_reorder(w, v, vt)
-    S64 = oracle.tile_scores(w, oracle.tile_pool(w, qp), oracle.tile_pool(w, kp))
+    S64 = oracle.block_scores(w, oracle.tile_pool(w, qp), oracle.tile_pool(w, kp))
     kept = oracle.kept_mask(w, oracle.select_topk(w, S64))
     tiles = list(range(0, g.NT, tile_stride)) + list(range(g.NT, g.NQ))
     oracle.attention(w, qp, kp, vp, kept, q_tiles=tiles)
@@ -217,14 +218,14 @@ def run_reference(args):
     import numpy as np
     import oracle
     import ssta_inputs as si
-    w = si.get_workload(args.workload)
+    w = workload_of(args)
     wh = si.with_overrides(w, H=1)
     g = oracle.geometry(wh)
     x = cpu_inputs(w, w.seeds[0], (0,))
     conv = lambda t: None if t is None else t.float().numpy().astype(np.float64)
     t0 = time.perf_counter()
     qp, kp, vp = (oracle.tile_reorder(wh, conv(x[n]), conv(x[n + "_text"])) for n in ("q", "k", "v"))
-    kept = oracle.kept_mask(wh, oracle.select_topk(wh, oracle.tile_scores(
+    kept = oracle.kept_mask(wh, oracle.select_topk(wh, oracle.block_scores(
         wh, oracle.tile_pool(wh, qp), oracle.tile_pool(wh, kp))))
     mask_s = time.perf_counter() - t0
     rng = np.random.default_rng(0)
@@ -264,6 +265,15 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU arm
+def workload_of(args):
+    """The named workload with the mask-mode flags applied."""
+    import ssta_inputs as si
+    w = si.get_workload(args.workload)
+    ov = {k: v for k, v in (("score_mode", args.score_mode), ("combine", args.combine),
+                            ("window_mode", args.window_mode)) if v is not None}
+    return si.with_overrides(w, **ov) if ov else w
+
+
 def rank_seeds(rank, base_seeds):
     """Weak scaling: rank r solves its own independent problems, seeds r*1000 + s."""
     return [rank * 1000 + s for s in base_seeds]
@@ -306,7 +316,7 @@ def run_gpu(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    w = si.get_workload(args.workload)
+    w = workload_of(args)
     d = S.desc_from(w)
     plan = S.ssta_plan(d)
     seeds = rank_seeds(rank, w.seeds)
@@ -467,6 +477,7 @@ def run_gpu(args):
             "config": {"workload": w.name, "B": w.B, "heads": w.H, "head_dim": w.D,
                        "grid": [w.T, w.Y, w.X], "tile": [w.tT, w.tY, w.tX], "window": [w.wT, w.wY, w.wX],
                        "topk": w.topk, "text_tokens": w.L_text, "seeds_per_rank": seeds,
+                       "mask": {"score": w.score_mode, "combine": w.combine, "window": w.window_mode},
                        "parallelism": f"dp{world} (one independent problem per rank)",
                        "l2": "no flush: every input tensor (0.9-1.0 GB) is larger than the 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": "ssta_attention_tc_kernel", "achieved": achieved,
@@ -487,7 +498,7 @@ def run_gpu(args):
                     "ms_per_step": max_e2e_ms / args.steps,
                     "copies": "pinned host buffers; uploads and downloads on two copy streams, overlapped with "
                               "the previous/next step's compute through double-buffered device inputs and outputs"},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": (LAUNCHES_PER_STEP + (2 if w.score_mode == "importance" else 0)) * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
@@ -506,6 +517,10 @@ def main():
     ap.add_argument("--impl", default="ssta", choices=["ssta", "reference"])
     ap.add_argument("--workload", default="p720_10s_bf16")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--score-mode", default=None, choices=["similarity", "importance"],
+                    help="block score ranked by top-k (default: the workload's, similarity)")
+    ap.add_argument("--combine", default=None, choices=["union", "and"])
+    ap.add_argument("--window-mode", default=None, choices=["shift", "truncate"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -70,7 +70,7 @@ ssta_status make_geom(const ssta_desc* d, Geom* g) {
   x.lambda = d->score_mode == SSTA_SCORE_IMPORTANCE ? d->lambda : 0.0f;
   x.combine = d->combine;
   x.window_mode = d->window_mode;
-  x.norm_blocks = ceil_div(x.NT, 128);
+  x.norm_blocks = ceil_div(x.NT, 32);
   *g = x;
   return SSTA_OK;
 }
@@ -146,12 +146,11 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(w + ws.scores);
   const bool imp = g.score_mode == SSTA_SCORE_IMPORTANCE;
   const ImportanceBufs ib = imp ? ImportanceBufs{reinterpret_cast<float*>(w + ws.inv_nq), reinterpret_cast<float*>(w + ws.inv_nk),
-                                                 reinterpret_cast<float*>(w + ws.ksum), reinterpret_cast<float*>(w + ws.red)}
-                                : ImportanceBufs{nullptr, nullptr, nullptr, nullptr};
+                                                 reinterpret_cast<float*>(w + ws.ksum)}
+                                : ImportanceBufs{nullptr, nullptr, nullptr};
   // the pool kernel also clears the status word
-  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(w + ws.status), s);
-  if (e == cudaSuccess && imp) e = launch_tile_norms(g, qbar, kbar, ib, s);
-  if (e == cudaSuccess && imp) e = launch_tile_redundancy(g, kbar, ib, s);
+  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(w + ws.status), ib, s);
+  if (e == cudaSuccess && imp) e = launch_tile_keysum(g, kbar, ib, s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return from_cuda(e);

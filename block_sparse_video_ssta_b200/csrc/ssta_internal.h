@@ -32,7 +32,7 @@ struct Geom {
   float lambda;         // importance score weight
   int combine;          // ssta_combine
   int window_mode;      // ssta_window
-  int norm_blocks;      // 128-tile blocks of the importance pre-pass = ceil(NT/128)
+  int norm_blocks;      // 32-tile blocks of the importance key sums = ceil(NT/32)
 };
 
 // Workspace layout of ssta_build_block_mask (byte offsets, 256-aligned).
@@ -42,8 +42,7 @@ struct MaskWorkspace {
   size_t kbar;     // fp32 [BH, D, NT] (channel-major)
   size_t inv_nq;   // importance score only: fp32 [BH, NT], 1 / |Qbar_i| (0 for a zero mean)
   size_t inv_nk;   //   fp32 [BH, NT], 1 / |Kbar_j|
-  size_t ksum;     //   fp32 [BH, norm_blocks, D], per 128-tile block sum of unit Kbar_j
-  size_t red;      //   fp32 [BH, NT], redundancy of key tile j
+  size_t ksum;     //   fp32 [BH, norm_blocks, D], per 32-tile block sum of unit Kbar_j
   size_t scores;   // fp32 [BH, NT, NT]; absent when `with_scores` is false
   size_t total;
 };
@@ -56,7 +55,6 @@ struct ImportanceBufs {
   float* inv_nq;
   float* inv_nk;
   float* ksum;
-  float* red;
 };
 
 // Validate a descriptor and derive every size (host only, no CUDA call).
@@ -68,15 +66,13 @@ cudaError_t launch_tile_reorder(const Geom& g, const void* raster, const void* t
 cudaError_t launch_tile_unorder(const Geom& g, const void* packed, void* raster, void* text,
                                 cudaStream_t s);
 // Also writes 0 to *status (when non-NULL) after the previous kernel of the stream has
-// finished, so a mask build needs no separate reset of its status word.
+// finished, so a mask build needs no separate reset of its status word, and, for the
+// importance score (ib.inv_nq != NULL), the inverse norms of the tile means.
 cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, float* qbar, float* kbar,
-                             int32_t* status, cudaStream_t s);
-// Importance score only: per-tile inverse norms and per-block sums of unit key means,
-// then the per-key redundancy.  Both wait for the previous kernel (programmatic launch).
-cudaError_t launch_tile_norms(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
-                              cudaStream_t s);
-cudaError_t launch_tile_redundancy(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s);
-// Block scores: raw dot products, or the importance score when ib.red != NULL.
+                             int32_t* status, const ImportanceBufs& ib, cudaStream_t s);
+// Importance score only: per 32-tile block sums of the unit key means.
+cudaError_t launch_tile_keysum(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s);
+// Block scores: raw dot products, or the importance score when ib.ksum != NULL.
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
                                float* scores, cudaStream_t s);
 cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,

@@ -11,15 +11,16 @@
 //                         valid q and k rows with 16-byte coalesced loads and
 //                         reduces per-channel fp32 sums across row groups; the
 //                         means are stored channel-major for the score kernel.
-//   tile_norms_kernel,    importance score only: inverse norms of the tile
-//   tile_redundancy_kernel means and the per-key redundancy (mean key-key
-//                         similarity to the other key tiles), O(NT*D) per head
-//                         through the sum of the unit key means.
+//   tile_keysum_kernel    importance score only: per 32-tile block sums of the
+//                         unit key means (the pool kernel writes the norms);
+//                         the score kernel turns them into each key tile's
+//                         redundancy (mean key-key similarity to the other key
+//                         tiles) in O(NT*D) per head, without an NT x NT product.
 //   tile_scores_kernel    fp32 SIMT, 128x128 score blocks per CTA, 8x8 per
 //                         thread, 16-channel stages double-buffered in shared
 //                         memory by cp.async, channels summed in order 0..D-1
 //                         with FMA (packed f32x2, two columns per instruction);
-//                         the importance transform is applied in the epilogue.
+//                         the importance score is formed in the epilogue.
 //   select_and_list_kernel one warp per (head, query tile): top-k over scores
 //                         held in registers as order-preserving 32-bit keys
 //                         (bitwise binary search for the k-th key with warp-wide
@@ -79,7 +80,7 @@ __device__ __forceinline__ void add_vec(float* acc, const int4& raw, const float
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ kp,
-                 float* __restrict__ qbar, float* __restrict__ kbar, int32_t* __restrict__ status) {
+                 float* __restrict__ qbar, float* __restrict__ kbar, int32_t* __restrict__ status, ImportanceBufs ib) {
   allow_dependents();
   grid_dependency_wait();   // q and k are packed by the previous kernels
   if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
@@ -140,82 +141,57 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
   }
   __syncthreads();
   const float inv = 1.0f / (float)(vt * vy * vx);
+  float sq[2] = {0.f, 0.f};   // squares of this thread's means, for q and for k
   for (int t = threadIdx.x; t < 2 * D; t += kPoolThreads) {
     const int which = t / D, ch = t % D;
     float s = 0.f;
     for (int r = 0; r < rpp; ++r) s += red[(which * rpp + r) * D + ch];
     float* out = which ? kbar : qbar;
-    out[(bh * D + ch) * g.NT + c] = s * inv;     // channel-major: [head][channel][tile]
+    const float mean = s * inv;
+    out[(bh * D + ch) * g.NT + c] = mean;     // channel-major: [head][channel][tile]
+    sq[which] = fmaf(mean, mean, sq[which]);
   }
-}
-
-// Step 2, importance score, pre-pass 1 (one CTA per 128 tiles of one head, one
-// thread per tile): the inverse L2 norm of each tile mean of q and of k (0 for an
-// all-zero mean), and this block's sum of the unit-length key means, one value per
-// channel, reduced in a fixed order (warp shuffle tree, then the four warps in
-// order) so the result does not depend on scheduling.
-__global__ void __launch_bounds__(128)
-tile_norms_kernel(Geom g, const float* __restrict__ qbar_t, const float* __restrict__ kbar_t, ImportanceBufs ib) {
-  allow_dependents();
-  grid_dependency_wait();   // the pooled means are written by the previous kernel
-  __shared__ float part[4][128];
-  const int64_t bh = blockIdx.y;
-  const int NT = g.NT, D = g.D;
-  const int c = blockIdx.x * 128 + threadIdx.x;
-  const bool valid = c < NT;
-  const float* qh = qbar_t + bh * D * (int64_t)NT;
-  const float* kh = kbar_t + bh * D * (int64_t)NT;
-  float sq = 0.f, sk = 0.f;
-  if (valid) {
-    for (int d = 0; d < D; ++d) {
-      const float a = qh[(int64_t)d * NT + c], b = kh[(int64_t)d * NT + c];
-      sq = fmaf(a, a, sq);
-      sk = fmaf(b, b, sk);
+  if (ib.inv_nq != nullptr) {
+    // importance score: 1 / |mean| of q and of k (0 for an all-zero mean), fixed-order reduction
+    __shared__ float nsq[2][kPoolThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      float v = sq[which];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+      if (lane == 0) nsq[which][warp] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < 2) {
+      float a = 0.f;
+      for (int w = 0; w < kPoolThreads / 32; ++w) a += nsq[threadIdx.x][w];
+      (threadIdx.x ? ib.inv_nk : ib.inv_nq)[bh * g.NT + c] = a > 0.f ? 1.0f / sqrtf(a) : 0.f;
     }
   }
-  const float iq = sq > 0.f ? 1.0f / sqrtf(sq) : 0.f;
-  const float ik = sk > 0.f ? 1.0f / sqrtf(sk) : 0.f;
-  if (valid) {
-    ib.inv_nq[bh * NT + c] = iq;
-    ib.inv_nk[bh * NT + c] = ik;
-  }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int d = 0; d < D; ++d) {
-    float v = valid ? kh[(int64_t)d * NT + c] * ik : 0.f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
-    if (lane == 0) part[warp][d] = v;
-  }
-  __syncthreads();
-  for (int d = threadIdx.x; d < D; d += 128)
-    ib.ksum[(bh * g.norm_blocks + blockIdx.x) * D + d] = ((part[0][d] + part[1][d]) + part[2][d]) + part[3][d];
 }
 
-// Step 2, importance score, pre-pass 2 (same grid): the redundancy of key tile j,
-// the mean over the other key tiles j' of (u_j' . u_j + 1) / 2 with u the unit key
-// means, through sum_{j' != j} u_j' . u_j = (sum_j' u_j') . u_j - |u_j|^2; the
-// per-block sums are added in block order.  0 when the grid has one tile.
+// Step 2, importance score, pre-pass (one CTA per 32 key tiles of one head, one
+// thread per channel): this block's sum of the unit-length key means,
+// sum_j Kbar_j[d] / |Kbar_j| in tile order, for the redundancy term.
+constexpr int kKeySumTiles = 32;
+
 __global__ void __launch_bounds__(128)
-tile_redundancy_kernel(Geom g, const float* __restrict__ kbar_t, ImportanceBufs ib) {
+tile_keysum_kernel(Geom g, const float* __restrict__ kbar_t, ImportanceBufs ib) {
   allow_dependents();
-  grid_dependency_wait();   // the per-block key sums are written by the previous kernel
-  __shared__ float usum[128];
+  grid_dependency_wait();   // the means and norms are written by the previous kernel
   const int64_t bh = blockIdx.y;
-  const int NT = g.NT, D = g.D;
-  for (int d = threadIdx.x; d < D; d += 128) {
-    float a = 0.f;
-    for (int b = 0; b < g.norm_blocks; ++b) a += ib.ksum[(bh * g.norm_blocks + b) * D + d];
-    usum[d] = a;
-  }
+  const int NT = g.NT;
+  const int c0 = blockIdx.x * kKeySumTiles, c1 = min(c0 + kKeySumTiles, NT);
+  __shared__ float ik[kKeySumTiles];
+  if (threadIdx.x < kKeySumTiles) ik[threadIdx.x] = c0 + (int)threadIdx.x < NT ? ib.inv_nk[bh * NT + c0 + threadIdx.x] : 0.f;
   __syncthreads();
-  const int c = blockIdx.x * 128 + threadIdx.x;
-  if (c >= NT) return;
-  const float* kh = kbar_t + bh * D * (int64_t)NT;
-  float dot = 0.f;
-  for (int d = 0; d < D; ++d) dot = fmaf(kh[(int64_t)d * NT + c], usum[d], dot);
-  const float ik = ib.inv_nk[bh * NT + c];
-  const float self = ik > 0.f ? 1.0f : 0.f;             // |u_j|^2
-  ib.red[bh * NT + c] = NT > 1 ? 0.5f + (dot * ik - self) / (2.0f * (float)(NT - 1)) : 0.f;
+  for (int d = threadIdx.x; d < g.D; d += 128) {
+    const float* row = kbar_t + (bh * g.D + d) * (int64_t)NT;
+    float a = 0.f;
+    for (int c = c0; c < c1; ++c) a = fmaf(row[c], ik[c - c0], a);
+    ib.ksum[(bh * g.norm_blocks + blockIdx.x) * g.D + d] = a;
+  }
 }
 
 // Step 2, Score_s = Qbar Kbar^T.  One CTA computes a 128 x 128 block of scores
@@ -304,6 +280,19 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
   const int nst = g.D / kScoreStage;
   allow_dependents();
   grid_dependency_wait();   // the pooled means are written by the previous kernel
+  // importance score: u = sum of the unit key means of the head (partial sums added in
+  // block order), and Kbar_j . u for this CTA's 128 key tiles, accumulated from the
+  // staged key means by two threads per tile (channels 0-7 and 8-15 of each stage)
+  const bool imp = ib.ksum != nullptr;
+  __shared__ float u_s[128], kd_s[2][kScoreBlock], red_s[kScoreBlock];
+  float kd = 0.f;
+  if (imp) {
+    for (int d = threadIdx.x; d < g.D; d += 256) {
+      float a = 0.f;
+      for (int b = 0; b < g.norm_blocks; ++b) a += ib.ksum[(bh * g.norm_blocks + b) * g.D + d];
+      u_s[d] = a;
+    }
+  }
   score_stage_copy<kVec>(qs[0], ks[0], qh, kh, NT, i0, j0, 0);
   cp_async_commit();
   for (int st = 0; st < nst; ++st) {
@@ -332,18 +321,34 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
         for (int b = 0; b < 4; ++b) acc[a][b] = f2_fma(q2, k2[b], acc[a][b]);
       }
     }
+    if (imp) {
+      const int cc = threadIdx.x & 127, c8 = (threadIdx.x >> 7) * 8;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) kd = fmaf(ks[buf][c8 + c][cc], u_s[st * kScoreStage + c8 + c], kd);
+    }
     __syncthreads();   // every thread is done with buffer buf before it is refilled
   }
   float* sh = scores + bh * NT * (int64_t)NT;
-  // importance score: lambda (cos + 1) / 2 - (1 - lambda) red_j, cos = dot / (|Qbar_i| |Kbar_j|)
-  const bool imp = ib.red != nullptr;
+  // importance score: lambda (cos + 1) / 2 - (1 - lambda) red_j with cos = dot / (|Qbar_i| |Kbar_j|)
+  // and red_j = the mean over j' != j of (u_j' . u_j + 1) / 2 (u = unit key means),
+  // through sum_{j' != j} u_j' . u_j = (sum_j' u_j') . u_j - |u_j|^2 (0 when NT = 1)
   float ck[8], rk[8];
   if (imp) {
+    kd_s[threadIdx.x >> 7][threadIdx.x & 127] = kd;
+    __syncthreads();
+    if (threadIdx.x < kScoreBlock) {
+      const int j = j0 + (int)threadIdx.x;
+      const float ik = j < NT ? ib.inv_nk[bh * NT + j] : 0.f;
+      const float self = ik > 0.f ? 1.0f : 0.f;
+      const float dot = (kd_s[0][threadIdx.x] + kd_s[1][threadIdx.x]) * ik;
+      red_s[threadIdx.x] = NT > 1 ? 0.5f + (dot - self) / (2.0f * (float)(NT - 1)) : 0.f;
+    }
+    __syncthreads();
 #pragma unroll
     for (int b = 0; b < 8; ++b) {
-      const int j = j0 + (b < 4 ? 4 * tx + b : 64 + 4 * tx + b - 4);
+      const int jj = b < 4 ? 4 * tx + b : 64 + 4 * tx + b - 4, j = j0 + jj;
       ck[b] = j < NT ? ib.inv_nk[bh * NT + j] : 0.f;
-      rk[b] = j < NT ? (1.0f - g.lambda) * ib.red[bh * NT + j] : 0.f;
+      rk[b] = (1.0f - g.lambda) * red_s[jj];
     }
   }
 #pragma unroll
@@ -411,7 +416,8 @@ __device__ __forceinline__ uint32_t range_bits(int word, int lo, int hi) {
 //    32-tile words, followed by the text tiles and -1 padding.
 // Text query tiles keep every tile.
 constexpr int kBucketCap = 64;
-constexpr int kHiBits = 12;   // prefix bits searched over every key
+constexpr int kHiBits = 12;       // prefix bits searched over every key
+constexpr int kHiBitsWide = 16;   // ... when the 12-bit bucket holds more than kBucketCap keys
 
 template <int SLOTS>
 __global__ void __launch_bounds__(256)
@@ -441,16 +447,19 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
     for (int q = 0; q < (SLOTS + 31) / 32; ++q) myword[q] = 0u;
     const int k = g.k;
     if (k > 0) {
-      // k-th largest key in two levels: a bitwise search over the upper kHiBits bits of
-      // every key, then over the remaining low bits of the keys that share the found
-      // prefix (the boundary bucket, compacted into shared memory when it holds at most
-      // 64; otherwise the low bits are searched over all keys).  `above` = number of
-      // keys whose prefix is larger, i.e. the count of the last candidate that failed.
-      constexpr int kLoBits = 32 - kHiBits;
+      // k-th largest key in two levels: a bitwise search over the upper 12 bits of every
+      // key (16 when more than 64 keys share the found 12-bit prefix, as for scores
+      // packed into a narrow range), then over the remaining low bits of the keys that
+      // share the found prefix (the boundary bucket, compacted into shared memory when
+      // it holds at most 64; otherwise the low bits are searched over all keys).
+      // `above` = keys whose prefix is larger (the count of the last candidate that
+      // failed); `at_or_above` = keys whose prefix is at least the found one (the count
+      // of the last candidate that passed).
       uint32_t hi = 0;
-      int above = 0;
-      for (int bit = kHiBits - 1; bit >= 0; --bit) {
-        const uint32_t cand = (hi | (1u << bit)) << kLoBits;
+      int above = 0, at_or_above = g.NT;
+      int hi_bits = kHiBits;
+      for (int bit = 31; bit >= 32 - hi_bits; --bit) {
+        const uint32_t cand = (hi | (1u << bit));
         int c0 = 0, c1 = 0;
 #pragma unroll
         for (int w = 0; w < SLOTS; w += 2) {
@@ -458,14 +467,21 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
           if (w + 1 < SLOTS) c1 += (key[w + 1] >= cand) ? 1 : 0;
         }
         const int cnt = __reduce_add_sync(0xffffffffu, c0 + c1);
-        if (cnt >= k) hi |= 1u << bit;
-        else above = cnt;
+        if (cnt >= k) {
+          hi = cand;
+          at_or_above = cnt;
+        } else {
+          above = cnt;
+        }
+        if (bit == 32 - kHiBits && hi_bits == kHiBits && at_or_above - above > kBucketCap) hi_bits = kHiBitsWide;
       }
+      const int lo_bits = 32 - hi_bits;
+      hi >>= lo_bits;
       int bsize = 0;
       uint32_t* bucket = bucket_smem + (threadIdx.x >> 5) * kBucketCap;
 #pragma unroll
       for (int w = 0; w < SLOTS; ++w) {
-        const bool in = key[w] != 0u && (key[w] >> kLoBits) == hi;
+        const bool in = key[w] != 0u && (key[w] >> lo_bits) == hi;
         const uint32_t m = __ballot_sync(0xffffffffu, in);
         if (m) {   // warp-uniform; most slots hold no key of the bucket
           const int pos = bsize + __popc(m & lt_mask);
@@ -475,17 +491,17 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
       }
       __syncwarp();
       const int need_lo = k - above;     // keys to take from the bucket (>= 1)
-      uint32_t thr = hi << kLoBits;
+      uint32_t thr = hi << lo_bits;
       if (bsize <= kBucketCap) {
         const uint32_t b0 = lane < bsize ? bucket[lane] : 0u;
         const uint32_t b1 = lane + 32 < bsize ? bucket[lane + 32] : 0u;
-        for (int bit = kLoBits - 1; bit >= 0; --bit) {
+        for (int bit = lo_bits - 1; bit >= 0; --bit) {
           const uint32_t cand = thr | (1u << bit);
           const int cnt = __reduce_add_sync(0xffffffffu, (b0 >= cand ? 1 : 0) + (b1 >= cand ? 1 : 0));
           if (cnt >= need_lo) thr = cand;
         }
       } else {
-        for (int bit = kLoBits - 1; bit >= 0; --bit) {
+        for (int bit = lo_bits - 1; bit >= 0; --bit) {
           const uint32_t cand = thr | (1u << bit);
           int cnt = 0;
 #pragma unroll
@@ -598,8 +614,7 @@ MaskWorkspace mask_workspace_layout(const Geom& g, bool with_scores) {
     w.inv_nq = end;
     w.inv_nk = w.inv_nq + up(bh * g.NT * sizeof(float));
     w.ksum = w.inv_nk + up(bh * g.NT * sizeof(float));
-    w.red = w.ksum + up(bh * g.norm_blocks * g.D * sizeof(float));
-    end = w.red + up(bh * g.NT * sizeof(float));
+    end = w.ksum + up(bh * g.norm_blocks * g.D * sizeof(float));
   }
   w.scores = end;
   w.total = end + (with_scores ? up(bh * g.NT * (size_t)g.NT * sizeof(float)) : 0);
@@ -607,7 +622,7 @@ MaskWorkspace mask_workspace_layout(const Geom& g, bool with_scores) {
 }
 
 cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, float* qbar, float* kbar,
-                             int32_t* status, cudaStream_t s) {
+                             int32_t* status, const ImportanceBufs& ib, cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
   dim3 grid(g.NT, g.B * g.H);
   const int epv = 16 / g.esize;
@@ -617,20 +632,14 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
   const int4* k4 = static_cast<const int4*>(kp);
   if (g.dtype == SSTA_BF16)
     return launch_dependent(tile_pool_kernel<__nv_bfloat16>, grid, dim3(kPoolThreads), smem, s, g, q4, k4, qbar,
-                            kbar, status);
+                            kbar, status, ib);
   return launch_dependent(tile_pool_kernel<float>, grid, dim3(kPoolThreads), smem, s, g, q4, k4, qbar, kbar,
-                          status);
+                          status, ib);
 }
 
-cudaError_t launch_tile_norms(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
-                              cudaStream_t s) {
+cudaError_t launch_tile_keysum(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
-  return launch_dependent(tile_norms_kernel, dim3(g.norm_blocks, g.B * g.H), dim3(128), 0, s, g, qbar, kbar, ib);
-}
-
-cudaError_t launch_tile_redundancy(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s) {
-  if ((int64_t)g.B * g.H == 0) return cudaSuccess;
-  return launch_dependent(tile_redundancy_kernel, dim3(g.norm_blocks, g.B * g.H), dim3(128), 0, s, g, kbar, ib);
+  return launch_dependent(tile_keysum_kernel, dim3(g.norm_blocks, g.B * g.H), dim3(128), 0, s, g, kbar, ib);
 }
 
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,

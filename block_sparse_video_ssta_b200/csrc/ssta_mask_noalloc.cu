@@ -83,12 +83,11 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(base + ws.scores);
   const bool imp = g.score_mode == SSTA_SCORE_IMPORTANCE;
   const ImportanceBufs ib = imp ? ImportanceBufs{reinterpret_cast<float*>(base + ws.inv_nq), reinterpret_cast<float*>(base + ws.inv_nk),
-                                                 reinterpret_cast<float*>(base + ws.ksum), reinterpret_cast<float*>(base + ws.red)}
-                                : ImportanceBufs{nullptr, nullptr, nullptr, nullptr};
+                                                 reinterpret_cast<float*>(base + ws.ksum)}
+                                : ImportanceBufs{nullptr, nullptr, nullptr};
   // the pool kernel also clears the status word
-  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(base + ws.status), s);
-  if (e == cudaSuccess && imp) e = launch_tile_norms(g, qbar, kbar, ib, s);
-  if (e == cudaSuccess && imp) e = launch_tile_redundancy(g, kbar, ib, s);
+  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(base + ws.status), ib, s);
+  if (e == cudaSuccess && imp) e = launch_tile_keysum(g, kbar, ib, s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;

@@ -108,7 +108,7 @@ def compare_attention(w, O_gpu, lse_gpu, O_ref, lse_ref, rows_mask):
     rel = float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
     la, lb = lse_gpu[rows_mask], lse_ref[rows_mask]
     empty = np.isneginf(la) & np.isneginf(lb)                 # rows with no kept key on both sides
-    lse_err = float(np.where(empty, 0.0, np.abs(la - lb)).max()) if err.size else 0.0
+    lse_err = float(np.abs(np.where(empty, 0.0, la) - np.where(empty, 0.0, lb)).max()) if err.size else 0.0
     assert max_abs <= tol["o_max"], f"O max-abs {max_abs} > {tol['o_max']}"
     assert rel <= tol["o_rel"], f"O rel-L2 {rel} > {tol['o_rel']}"
     assert lse_err <= tol["lse_max"], f"LSE max-abs {lse_err} > {tol['lse_max']}"

@@ -60,7 +60,7 @@ import numpy as np
 __all__ = [
     "Geometry", "geometry", "valid_token_mask", "tile_reorder", "tile_unorder",
     "tile_pool", "tile_scores", "importance_scores", "block_scores", "select_topk", "window_mask", "kept_mask",
-    "kept_lists", "attention", "ssta_forward", "attention_flops",
+    "kept_lists", "attention", "attention_bwd", "ssta_forward", "attention_flops",
 ]
 
 
@@ -324,6 +324,48 @@ def attention(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, kept: np.ndarra
                 O[b, h, r0:r1] = p @ v[keys]
                 LSE[b, h, r0:r1] = lse
     return O, LSE
+
+
+def attention_bwd(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, dOp: np.ndarray, kept: np.ndarray,
+                  scale: float | None = None):
+    """Gradients of Step 4's block-sparse attention, in float64: for every valid
+    query row of query tile i and the valid keys of its kept tiles, with
+    P = softmax(q k^T * scale) (recomputed), O = P v, D = rowsum(dO * O):
+    dS = P * (dO v^T - D), dQ = scale * dS k, dK += scale * dS^T q, dV += P^T dO.
+    Pad query rows take no part (their dQ is 0); pad keys get dK = dV = 0; a query
+    tile with no kept key contributes nothing.  Returns (dQ, dK, dV), each
+    [B,H,Lq,D] on the packed layout."""
+    g = geometry(d)
+    scale = 1.0 / math.sqrt(g.D) if not scale else scale
+    B, H = qp.shape[:2]
+    valid = valid_token_mask(d)
+    dQ = np.zeros((B, H, g.Lq, g.D))
+    dK = np.zeros((B, H, g.Lq, g.D))
+    dV = np.zeros((B, H, g.Lq, g.D))
+    for b in range(B):
+        for h in range(H):
+            q = qp[b, h].astype(np.float64)
+            k = kp[b, h].astype(np.float64)
+            v = vp[b, h].astype(np.float64)
+            do = dOp[b, h].astype(np.float64)
+            for i in range(g.NQ):
+                r0, r1 = i * g.N, min((i + 1) * g.N, g.Lq)
+                rows = np.arange(r0, r1)[valid[r0:r1]]
+                cols = [np.arange(j * g.N, min((j + 1) * g.N, g.Lq)) for j in np.nonzero(kept[b, h, i])[0]]
+                keys = np.concatenate([c[valid[c]] for c in cols]) if cols else np.zeros(0, dtype=np.int64)
+                if keys.size == 0 or rows.size == 0:
+                    continue
+                s = (q[rows] @ k[keys].T) * scale
+                m = s.max(axis=1, keepdims=True)
+                p = np.exp(s - m)
+                p /= p.sum(axis=1, keepdims=True)
+                o = p @ v[keys]
+                Dr = (do[rows] * o).sum(axis=1, keepdims=True)
+                ds = p * (do[rows] @ v[keys].T - Dr)
+                dQ[b, h, rows] = scale * ds @ k[keys]
+                np.add.at(dK[b, h], keys, scale * ds.T @ q[rows])
+                np.add.at(dV[b, h], keys, p.T @ do[rows])
+    return dQ, dK, dV
 
 
 def attention_flops(d, kept: np.ndarray, padded: bool = True) -> float:

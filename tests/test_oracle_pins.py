@@ -20,7 +20,10 @@
   scaling of the pooled vectors, lambda = 1 reducing to (cosine + 1) / 2, a
   single tile and all-zero vectors; top-k on them by brute force;
 * truncated window: brute force over each axis and the pages' |c' - c| <= w/2
-  rule; AND combination: set intersection, and its two degenerate cases.
+  rule; AND combination: set intersection, and its two degenerate cases;
+* backward (dQ, dK, dV): torch autograd through the float64 masked SDPA on the
+  raster tokens (random kept sets with and without text, the dense case), the
+  invariants sum_keys dV = sum_rows dO and sum_keys dK = 0, empty kept sets.
 
 Sources: "HunyuanVideo 1.5 Technical Report" (paper-graph-ui summary),
 section "SSTA: Selective and Sliding Tile Attention", Steps 1-4 and the
@@ -522,3 +525,87 @@ def test_empty_kept_set_gives_zero_output():
     O, L = oracle.attention(w, qp, kp, vp, kept)
     assert np.all(O[:, :, g.N:] == 0.0) and np.all(np.isneginf(L[:, :, g.N:]))
     assert np.all(np.isfinite(L[:, :, : g.N]))
+
+
+# ---------------------------------------------------------------------------
+# Backward of Step 4: dQ, dK, dV
+# ---------------------------------------------------------------------------
+
+def _sdpa_grads(d, arrs, dO_raster, dO_text, allowed):
+    """torch autograd (float64) through the masked SDPA on raster tokens [+ text]."""
+    q, k, v, qt, kt, vt = arrs
+    B, H = q.shape[:2]
+    L = d.T * d.Y * d.X
+    cat = lambda a, b: np.concatenate([a.reshape(B, H, L, d.D)] + ([b] if b is not None else []), axis=2)
+    Q, K, V = (torch.from_numpy(cat(a, b)).requires_grad_(True) for a, b in ((q, qt), (k, kt), (v, vt)))
+    O = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=torch.from_numpy(allowed))
+    (O * torch.from_numpy(cat(dO_raster, dO_text))).sum().backward()
+    return Q.grad.numpy(), K.grad.numpy(), V.grad.numpy()
+
+
+def _bwd_case(d, seed, kept_fn):
+    g = oracle.geometry(d)
+    x = si.make_inputs(d, seed)
+    arrs, r = _run_oracle(d, x)
+    kept = kept_fn(d, g, r)
+    rng = np.random.default_rng(seed + 100)
+    dO_r = rng.standard_normal((d.B, d.H, d.T, d.Y, d.X, d.D))
+    dO_t = rng.standard_normal((d.B, d.H, d.L_text, d.D)) if d.L_text else None
+    dOp = oracle.tile_reorder(d, dO_r, dO_t)
+    dQ, dK, dV = oracle.attention_bwd(d, r["qp"], r["kp"], r["vp"], dOp, kept)
+    return g, arrs, r, kept, dO_r, dO_t, dOp, (dQ, dK, dV)
+
+
+def _to_raster(d, t):
+    B, H = t.shape[:2]
+    L = d.T * d.Y * d.X
+    ras, txt = oracle.tile_unorder(d, t)
+    return np.concatenate([ras.reshape(B, H, L, d.D)] + ([txt] if d.L_text else []), axis=2)
+
+
+@pytest.mark.parametrize("L_text", [0, 37])
+def test_backward_equals_autograd_random_kept(L_text):
+    d = with_overrides(_desc(T=4, Y=8, X=6, tT=2, tY=4, tX=3, L_text=L_text, H=2, D=8), recipe="tile_offset")
+
+    def kept_fn(d, g, r):
+        rng = np.random.default_rng(7)
+        kept = rng.random((d.B, d.H, g.NQ, g.NQ)) < 0.4
+        kept[:, :, np.arange(g.NQ), np.arange(g.NQ)] = True        # every row keeps something
+        return kept
+
+    g, arrs, r, kept, dO_r, dO_t, dOp, grads = _bwd_case(d, 11, kept_fn)
+    ref = _sdpa_grads(d, arrs, dO_r, dO_t, _token_mask_from_tile_mask(d, kept))
+    for got, want in zip(grads, ref):
+        np.testing.assert_allclose(_to_raster(d, got), want, rtol=0, atol=1e-11)
+    valid = oracle.valid_token_mask(d)
+    for t in grads:                                                    # pad rows stay zero
+        assert np.all(t[:, :, ~valid] == 0.0)
+
+
+def test_backward_dense_and_invariants():
+    d = si.get_workload("tiny_f32")
+    d = with_overrides(d, wT=9, wY=9, wX=9, topk=0, L_text=20)          # window = whole grid: dense
+
+    def kept_fn(d, g, r):
+        return r["kept"]
+
+    g, arrs, r, kept, dO_r, dO_t, dOp, (dQ, dK, dV) = _bwd_case(d, 12, kept_fn)
+    ref = _sdpa_grads(d, arrs, dO_r, dO_t, _token_mask_from_tile_mask(d, kept))
+    for got, want in zip((dQ, dK, dV), ref):
+        np.testing.assert_allclose(_to_raster(d, got), want, rtol=0, atol=1e-11)
+    valid = oracle.valid_token_mask(d)
+    # rows of P sum to 1: the dV of all keys sums to the dO of all valid query rows;
+    # rows of dS sum to 0: the dK of all keys sums to 0
+    np.testing.assert_allclose(dV.sum(axis=2), dOp[:, :, valid].sum(axis=2), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dK.sum(axis=2), 0.0, rtol=0, atol=1e-10)
+
+
+def test_backward_empty_rows_contribute_nothing():
+    d = with_overrides(si.get_workload("tiny_f32"), combine="and", wT=1, wY=1, wX=1, topk=0)
+
+    def kept_fn(d, g, r):
+        return r["kept"]                                                # nothing kept anywhere
+
+    g, arrs, r, kept, dO_r, dO_t, dOp, (dQ, dK, dV) = _bwd_case(d, 13, kept_fn)
+    assert not kept.any()
+    assert not dQ.any() and not dK.any() and not dV.any()

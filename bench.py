@@ -509,6 +509,56 @@ def run_gpu(args):
     return 0
 
 
+def run_backward(args):
+    """Time the backward (dQ, dK, dV) on one GPU: inputs, O, LSE, kept lists and dO resident;
+    effective TFLOP/s = 2.5 x the forward's kept-block FLOPs (five products instead of two)."""
+    import torch
+    import block_sparse_video_ssta_b200 as S
+    import ssta_inputs as si
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload_of(args)
+    d = S.desc_from(w)
+    plan = S.ssta_plan(d)
+    x = si.make_inputs(w, w.seeds[0], device=dev)
+    r = S.ssta_forward(d, x["q"], x["k"], x["v"], x["q_text"], x["k_text"], x["v_text"])
+    dO = torch.randn(r["O_packed"].shape, device=dev, generator=torch.Generator(device=dev).manual_seed(5)
+                     ).to(r["O_packed"].dtype)
+    outs = [torch.empty_like(dO) for _ in range(3)]
+    ws = torch.empty(plan.bwd_workspace_bytes, dtype=torch.uint8, device=dev)
+    call = lambda: S.ssta_attention_bwd(d, r["qp"], r["kp"], r["vp"], r["O_packed"], r["LSE"], dO,
+                                        r["kv_idx"], r["kv_cnt"], *outs, workspace=ws)
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    assert S.ssta_read_device_status(ws) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(pci_bus_id(dev)) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    fwd_flops, _ = kept_flops(w, plan, r["kv_idx"], r["kv_cnt"])
+    tflops = 2.5 * fwd_flops / (ms / 1000.0) / 1e12
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops_sustained"])
+    line = {
+        "metric": "SSTA bwd ms/call & effective TFLOPS (2.5x kept-block forward FLOPs)", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "pass": "backward", "grid": [w.T, w.Y, w.X], "heads": w.H,
+                   "mask": {"score": w.score_mode, "combine": w.combine, "window": w.window_mode},
+                   "kernels": "SIMT (fp32 arithmetic), not tensor cores"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                     "peak_source": f"{src} bf16_tflops_sustained", "traffic": None},
+        "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -521,9 +571,13 @@ def main():
                     help="block score ranked by top-k (default: the workload's, similarity)")
     ap.add_argument("--combine", default=None, choices=["union", "and"])
     ap.add_argument("--window-mode", default=None, choices=["shift", "truncate"])
+    ap.add_argument("--backward", action="store_true",
+                    help="time ssta_attention_bwd instead of the forward (prints its own line)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.backward:
+        return run_backward(args)
     return run_gpu(args)
 
 

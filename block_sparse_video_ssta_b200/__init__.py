@@ -18,7 +18,7 @@ import torch
 
 __all__ = [
     "SstaError", "SSTA_BF16", "SSTA_F32", "Desc", "desc_from", "ssta_plan", "ssta_tile_reorder",
-    "ssta_build_block_mask", "ssta_attention_fwd", "ssta_tile_unorder", "ssta_read_device_status",
+    "ssta_build_block_mask", "ssta_attention_fwd", "ssta_attention_bwd", "ssta_tile_unorder", "ssta_read_device_status",
     "ssta_status_string", "ssta_forward", "library_path", "lib",
 ]
 
@@ -27,7 +27,7 @@ _LIB_PATH = os.path.join(_HERE, "libssta.so")
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        f"{_LIB_PATH} is missing: build it with `python -m block_sparse_video_ssta_b200.build` "
+        f"{_LIB_PATH} is missing: build it with `python block_sparse_video_ssta_b200/build.py` "
         "(there is no fallback implementation)")
 
 lib = ctypes.CDLL(_LIB_PATH)
@@ -54,7 +54,7 @@ class _PlanInfo(ctypes.Structure):
     _fields_ = [("packed_len", ctypes.c_int64), ("num_tiles", ctypes.c_int), ("num_text_tiles", ctypes.c_int),
                 ("num_q_tiles", ctypes.c_int), ("tile_tokens", ctypes.c_int), ("topk", ctypes.c_int),
                 ("window_tiles", ctypes.c_int), ("max_kept", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t),
-                ("attn_workspace_bytes", ctypes.c_size_t)]
+                ("attn_workspace_bytes", ctypes.c_size_t), ("bwd_workspace_bytes", ctypes.c_size_t)]
 
 
 _P = ctypes.c_void_p
@@ -64,6 +64,7 @@ _sig = {
     "ssta_tile_reorder": [_D, _P, _P, _P, _P],
     "ssta_build_block_mask": [_D, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "ssta_attention_fwd": [_D, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "ssta_attention_bwd": [_D, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "ssta_tile_unorder": [_D, _P, _P, _P, _P],
     "ssta_read_device_status": [_P, _P, ctypes.POINTER(ctypes.c_int32)],
 }
@@ -134,6 +135,7 @@ class Plan:
     max_kept: int
     workspace_bytes: int
     attn_workspace_bytes: int
+    bwd_workspace_bytes: int
 
 
 def ssta_plan(desc: Desc) -> Plan:
@@ -248,6 +250,31 @@ def ssta_attention_fwd(desc: Desc, q_packed, k_packed, v_packed, kv_idx, kv_cnt,
         _ptr(workspace, "workspace", torch.uint8), ctypes.c_size_t(workspace.numel()),
         _stream(stream, dev))
     return o_packed, lse, workspace
+
+
+def ssta_attention_bwd(desc: Desc, q_packed, k_packed, v_packed, o_packed, lse, do_packed, kv_idx, kv_cnt,
+                       dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward of Step 4: returns (dq, dk, dv [B,H,Lq,D], workspace)."""
+    p = ssta_plan(desc)
+    dt = _torch_dtype(desc)
+    dev = q_packed.device
+    shp = (desc.B, desc.H, p.packed_len, desc.D)
+    dq = torch.empty(shp, dtype=dt, device=dev) if dq is None else dq
+    dk = torch.empty(shp, dtype=dt, device=dev) if dk is None else dk
+    dv = torch.empty(shp, dtype=dt, device=dev) if dv is None else dv
+    if workspace is None:
+        workspace = _workspace(p.bwd_workspace_bytes, dev)
+    _call(
+        "ssta_attention_bwd", dev, ctypes.byref(desc),
+        _ptr(q_packed, "q_packed", dt, shp), _ptr(k_packed, "k_packed", dt, shp), _ptr(v_packed, "v_packed", dt, shp),
+        _ptr(o_packed, "o_packed", dt, shp), _ptr(lse, "lse", torch.float32, shp[:3]),
+        _ptr(do_packed, "do_packed", dt, shp),
+        _ptr(kv_idx, "kv_idx", torch.int32, (desc.B, desc.H, p.num_q_tiles, p.max_kept)),
+        _ptr(kv_cnt, "kv_cnt", torch.int32, (desc.B, desc.H, p.num_q_tiles)),
+        _ptr(dq, "dq", dt, shp), _ptr(dk, "dk", dt, shp), _ptr(dv, "dv", dt, shp),
+        _ptr(workspace, "workspace", torch.uint8), ctypes.c_size_t(workspace.numel()),
+        _stream(stream, dev))
+    return dq, dk, dv, workspace
 
 
 def ssta_tile_unorder(desc: Desc, x_packed, x_raster=None, x_text=None, stream=None, want_text=True):

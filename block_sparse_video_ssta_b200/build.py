@@ -1,6 +1,6 @@
 """Build libssta.so in-tree with nvcc for sm_100a.
 
-    python -m block_sparse_video_ssta_b200.build [--verbose]
+    python block_sparse_video_ssta_b200/build.py [--verbose]   (does not import the package)
 
 Each .cu under csrc/ compiles to an object in parallel, then one shared
 library is linked next to this file (the CUDA runtime is linked statically, so

@@ -96,6 +96,7 @@ ssta_status ssta_plan(const ssta_desc* desc, ssta_plan_info* info) {
   info->max_kept = g.max_kept;
   info->workspace_bytes = mask_workspace_layout(g).total;
   info->attn_workspace_bytes = 256;
+  info->bwd_workspace_bytes = bwd_workspace_layout(g).total;
   return SSTA_OK;
 }
 
@@ -109,6 +110,29 @@ ssta_status ssta_tile_reorder(const ssta_desc* desc, const void* x_raster, const
   if (!empty && g.L_text > 0 && x_text == nullptr) return SSTA_ERR_INVALID_ARG;
   if (!aligned(x_raster, 16) || !aligned(x_text, 16) || !aligned(x_packed, 16)) return SSTA_ERR_ALIGNMENT;
   return from_cuda(launch_tile_reorder(g, x_raster, x_text, x_packed, static_cast<cudaStream_t>(stream)));
+}
+
+ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, const void* k_packed,
+                               const void* v_packed, const void* o_packed, const float* lse, const void* do_packed,
+                               const int32_t* kv_idx, const int32_t* kv_cnt, void* dq_packed, void* dk_packed,
+                               void* dv_packed, void* workspace, size_t workspace_bytes, void* stream) {
+  Geom g;
+  ssta_status st = make_geom(desc, &g);
+  if (st != SSTA_OK) return st;
+  const BwdWorkspace ws = bwd_workspace_layout(g);
+  if (workspace == nullptr || workspace_bytes < ws.total) return SSTA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return SSTA_ERR_ALIGNMENT;
+  const bool empty = (int64_t)g.B * g.H == 0;
+  const void* in[] = {q_packed, k_packed, v_packed, o_packed, lse, do_packed, kv_idx, kv_cnt, dq_packed, dk_packed,
+                      dv_packed};
+  for (const void* p : in) {
+    if (!empty && p == nullptr) return SSTA_ERR_INVALID_ARG;
+    if (!aligned(p, 16)) return SSTA_ERR_ALIGNMENT;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), s) != cudaSuccess) return SSTA_ERR_LAUNCH;
+  return from_cuda(launch_attention_bwd(g, q_packed, k_packed, v_packed, o_packed, lse, do_packed, kv_idx, kv_cnt,
+                                        dq_packed, dk_packed, dv_packed, workspace, s));
 }
 
 ssta_status ssta_tile_unorder(const ssta_desc* desc, const void* x_packed, void* x_raster, void* x_text,

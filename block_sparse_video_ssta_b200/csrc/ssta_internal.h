@@ -57,6 +57,16 @@ struct ImportanceBufs {
   float* ksum;
 };
 
+// Workspace layout of ssta_attention_bwd (byte offsets, 256-aligned).
+struct BwdWorkspace {
+  size_t status;   // int32 device status word
+  size_t rowdot;   // fp32 [BH, Lq], D = rowsum(dO * O)
+  size_t tcnt;     // int32 [BH, NQ], query tiles keeping each key tile
+  size_t tidx;     // int32 [BH, NQ, NQ], those query tiles, ascending
+  size_t total;
+};
+BwdWorkspace bwd_workspace_layout(const Geom& g);
+
 // Validate a descriptor and derive every size (host only, no CUDA call).
 ssta_status make_geom(const ssta_desc* d, Geom* g);
 
@@ -80,6 +90,9 @@ cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* 
 cudaError_t launch_attention_f32(const Geom& g, const float* qp, const float* kp, const float* vp,
                                  const int32_t* kv_idx, const int32_t* kv_cnt, float* o, float* lse,
                                  int32_t* status, cudaStream_t s);
+cudaError_t launch_attention_bwd(const Geom& g, const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* dO, const int32_t* kv_idx, const int32_t* kv_cnt,
+                                 void* dq, void* dk, void* dv, void* workspace, cudaStream_t s);
 cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* kp, const void* vp,
                                      const int32_t* kv_idx, const int32_t* kv_cnt, void* o, float* lse,
                                      int32_t* status, cudaStream_t s);

@@ -122,6 +122,7 @@ typedef struct {
   int max_kept;            /* row width of kv_idx */
   size_t workspace_bytes;  /* workspace for ssta_build_block_mask (>= 256) */
   size_t attn_workspace_bytes; /* workspace for ssta_attention_fwd (256) */
+  size_t bwd_workspace_bytes;  /* workspace for ssta_attention_bwd */
 } ssta_plan_info;
 
 /*
@@ -185,6 +186,25 @@ ssta_status ssta_attention_fwd(const ssta_desc* desc, const void* q_packed, cons
                                const void* v_packed, const int32_t* kv_idx, const int32_t* kv_cnt,
                                void* o_packed, float* lse, void* workspace, size_t workspace_bytes,
                                void* stream);
+
+/*
+ * ssta_attention_bwd — gradients of ssta_attention_fwd (Step 4) for training: with
+ * P = exp(q k^T * scale - LSE) over the valid keys of each query tile's kept tiles,
+ * D = rowsum(dO * O) and dS = P * (dO v^T - D):
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
+ * Pad query rows take no part (dQ = 0 there); pad key rows get dK = dV = 0.
+ *   q/k/v/o/do_packed [B,H,Lq,D] (read; o and lse as ssta_attention_fwd wrote them,
+ *   do = dL/dO), kv_idx/kv_cnt as ssta_build_block_mask wrote them (ascending lists
+ *   required), dq/dk/dv_packed [B,H,Lq,D] (written in full), all of `dtype`;
+ *   workspace >= info.bwd_workspace_bytes (status word, per-row D, and for every key
+ *   tile the list of query tiles keeping it).
+ * SIMT kernels (fp32 arithmetic); the products are not on the tensor cores.
+ */
+ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, const void* k_packed,
+                               const void* v_packed, const void* o_packed, const float* lse,
+                               const void* do_packed, const int32_t* kv_idx, const int32_t* kv_cnt,
+                               void* dq_packed, void* dk_packed, void* dv_packed, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /*
  * ssta_tile_unorder — inverse of ssta_tile_reorder: scatter packed rows back to

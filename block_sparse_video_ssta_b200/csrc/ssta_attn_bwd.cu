@@ -12,10 +12,11 @@
 //   bwd_transpose_kernel  for each key tile, the ascending list of query tiles
 //                         that keep it (one warp per key tile: a binary search
 //                         in every query tile's sorted list, ballots, prefix).
-//   bwd_dq_kernel         one warp per query row, walking its tile's kept list.
+//   bwd_dq_kernel         one warp per query row, walking its tile's kept list
+//                         (fp32; bf16 runs bwd_dq_tc_kernel on the tensor cores).
 //   bwd_dkdv_kernel       one warp per key row, walking the transposed list.
-// These are SIMT kernels (fp32 arithmetic, one lane per four channels): the
-// correct baseline of the backward; the products are not on the tensor cores.
+// The SIMT kernels use fp32 arithmetic, one lane per four channels; for bf16 the
+// dQ products run on the tensor cores, dK and dV do not yet.
 #include "ssta_internal.h"
 
 #include <cuda_bf16.h>
@@ -221,6 +222,11 @@ bwd_dkdv_kernel(Geom g, const T* __restrict__ qp, const T* __restrict__ kp, cons
 }
 
 template <typename T>
+constexpr bool kTensorCores = false;   // bf16: dQ runs on the tensor cores (ssta_attn_bwd_tc.cu)
+template <>
+constexpr bool kTensorCores<__nv_bfloat16> = true;
+
+template <typename T>
 cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dO, const int32_t* kv_idx, const int32_t* kv_cnt,
                              void* dq, void* dk, void* dv, const BwdWorkspace& ws, uint8_t* base, cudaStream_t s) {
@@ -236,8 +242,13 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
   const T* tO = static_cast<const T*>(dO);
   bwd_rowdot_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, static_cast<const T*>(o), tO, Dv);
   bwd_transpose_kernel<<<tb, kBwdWarps * 32, 0, s>>>(g, kv_idx, kv_cnt, tidx, tcnt, status);
-  bwd_dq_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, kv_idx, kv_cnt, static_cast<T*>(dq),
-                                                 status);
+  if (kTensorCores<T> && g.N % 128 == 0) {
+    const cudaError_t e = launch_attention_bwd_dq_tc(g, q, k, v, dO, lse, Dv, kv_idx, kv_cnt, dq, status, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    bwd_dq_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, kv_idx, kv_cnt, static_cast<T*>(dq),
+                                                   status);
+  }
   bwd_dkdv_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, tidx, tcnt, static_cast<T*>(dk),
                                                    static_cast<T*>(dv));
   return cudaGetLastError();

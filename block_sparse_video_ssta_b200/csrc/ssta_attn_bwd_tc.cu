@@ -1,0 +1,314 @@
+// Backward of Step 4 on the tensor cores, dQ part ("HunyuanVideo 1.5 Technical
+// Report", section "SSTA: Selective and Sliding Tile Attention", Step 4; the
+// attention equation softmax(Q K^T / sqrt(d_k)) V over the kept tiles):
+//   dQ = scale * dS K,  dS = P * (dO V^T - D),  P = exp(Q K^T * scale - LSE),
+// with LSE from the forward and D = rowsum(dO * O).
+//
+// One CTA owns 128 query rows of one query tile and walks the tile's kept list
+// in 128-key chunks.  Warp roles:
+//   warps 0-3  one thread per query row: P and dS from S and dP in tensor
+//              memory; dS (bf16) is written over S; epilogue dQ * scale
+//   warp  4    TMA producer: Q and dO once, then K and V chunks (2-stage rings)
+//   warp  5    TMEM allocator and tcgen05.mma issuer
+// Tensor memory: S (fp32, 128 columns; dS as bf16 over its first 64), dP
+// (128 columns), dQ accumulator (128 columns).
+// Per chunk j the MMA warp issues dQ += dS(j-1) K(j-1) (A = dS from tensor
+// memory, B = K in shared memory read MN-major), then S(j) = Q K(j)^T and
+// dP(j) = dO V(j)^T (both from shared memory).  The pipe executes in order, so
+// S(j) overwrites dS(j-1) only after dQ has read it.
+// Every wait is bounded (ssta_wait.cuh), as in the forward kernel.
+#include "ssta_tc_common.cuh"
+
+namespace ssta {
+namespace {
+
+using namespace wait;
+using namespace tc;
+
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kStages = 2;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffDO = kOffQ + kTileBytes;
+constexpr uint32_t kOffK = kOffDO + kTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr int kNumBars = 14;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemAlloc = kOffMisc + 64 + 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 1500000000ull;
+
+enum : int {
+  BAR_Q = 0, BAR_KFULL = 1, BAR_KEMPTY = 3, BAR_VFULL = 5, BAR_VEMPTY = 7,
+  BAR_SFULL = 9, BAR_DSREADY = 10, BAR_DQDONE = 11, BAR_DRAIN = 12
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Geom g,
+                 const ChunkTables tb, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
+                 const float* __restrict__ lse, const float* __restrict__ Dv, __nv_bfloat16* __restrict__ dq,
+                 int32_t* __restrict__ status, float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t sQ = base + kOffQ, sDO = base + kOffDO, sK = base + kOffK, sV = base + kOffV;
+  auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffMisc + 8);
+  const Ctl ctl{abort_flag, status, kTimeoutNs};
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: one 128-row block of a query tile; text query tiles first
+  const int blocks = g.N / 128;
+  const int64_t BH = (int64_t)g.B * g.H;
+  const int64_t text_units = BH * g.n_text * blocks;
+  int64_t u = blockIdx.x;
+  int64_t bh;
+  int qt, blk;
+  if (u < text_units) {
+    bh = u / ((int64_t)g.n_text * blocks);
+    const int rem = (int)(u - bh * g.n_text * blocks);
+    qt = g.NT + rem / blocks;
+    blk = rem % blocks;
+  } else {
+    u -= text_units;
+    bh = u / ((int64_t)g.NT * blocks);
+    const int rem = (int)(u - bh * g.NT * blocks);
+    qt = rem / blocks;
+    blk = rem % blocks;
+  }
+  const int qrow0 = qt * g.N + blk * 128;
+  const int64_t list_row = bh * g.NQ + qt;
+  int cnt = __ldg(kv_cnt + list_row);
+  if (cnt < 0 || cnt > g.max_kept) {
+    if (threadIdx.x == 0) atomicExch(status, (int)SSTA_ERR_DEVICE_BOUNDS);
+    cnt = cnt < 0 ? 0 : g.max_kept;
+  }
+  const int32_t* list = kv_idx + list_row * g.max_kept;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BAR_Q), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(BAR_KFULL + s), 1);
+      mbar_init(bar(BAR_KEMPTY + s), 1);
+      mbar_init(bar(BAR_VFULL + s), 1);
+      mbar_init(bar(BAR_VEMPTY + s), 1);
+    }
+    mbar_init(bar(BAR_SFULL), 1);
+    mbar_init(bar(BAR_DSREADY), 128);
+    mbar_init(bar(BAR_DQDONE), 1);
+    mbar_init(bar(BAR_DRAIN), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int e = 0; e < cnt; ++e) {
+      const int t = __ldg(list + e);
+      if (t < 0 || t >= g.NQ) { atomicExch(status, (int)SSTA_ERR_DEVICE_BOUNDS); break; }
+    }
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + 128, tDQ = tmem + 256;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int z = (int)bh;
+      mbar_expect_tx(bar(BAR_Q), 2 * kTileBytes);
+      for (int b = 0; b < 2; ++b) {
+        tma_load_3d(sQ + b * kBox, &tmQ, b * 64, qrow0, z, bar(BAR_Q));
+        tma_load_3d(sDO + b * kBox, &tmDO, b * 64, qrow0, z, bar(BAR_Q));
+      }
+      int nK[kStages] = {0, 0}, nV[kStages] = {0, 0};
+      const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool) -> bool {
+        const int s = j & 1;
+        const uint32_t ph = (uint32_t)((j >> 1) & 1);
+        const int krow = t * g.N + ch * kChunk;
+        if (!wait_bounded(bar(BAR_KEMPTY + s), ph ^ 1u, ctl)) return false;
+        mbar_expect_tx(bar(BAR_KFULL + s), kTileBytes);
+        tma_load_3d(sK + s * kTileBytes, &tmK, 0, krow, z, bar(BAR_KFULL + s));
+        tma_load_3d(sK + s * kTileBytes + kBox, &tmK, 64, krow, z, bar(BAR_KFULL + s));
+        ++nK[s];
+        if (!wait_bounded(bar(BAR_VEMPTY + s), ph ^ 1u, ctl)) return false;
+        mbar_expect_tx(bar(BAR_VFULL + s), kTileBytes);
+        tma_load_3d(sV + s * kTileBytes, &tmV, 0, krow, z, bar(BAR_VFULL + s));
+        tma_load_3d(sV + s * kTileBytes + kBox, &tmV, 64, krow, z, bar(BAR_VFULL + s));
+        ++nV[s];
+        return true;
+      });
+      if (n < 0) {
+        drain_wait(bar(BAR_Q), 0, kTimeoutNs);
+        for (int s = 0; s < kStages; ++s) {
+          if (nK[s] > 0) drain_wait(bar(BAR_KFULL + s), (uint32_t)((nK[s] - 1) & 1), kTimeoutNs);
+          if (nV[s] > 0) drain_wait(bar(BAR_VFULL + s), (uint32_t)((nV[s] - 1) & 1), kTimeoutNs);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const bool ok = wait_bounded(bar(BAR_Q), 0, ctl);
+      // dQ += dS(jp) K(jp): A = dS (bf16, columns 0..63 of S), B = K stage read MN-major
+      auto dq_step = [&](int jp) -> bool {
+        if (!wait_bounded(bar(BAR_DSREADY), (uint32_t)(jp & 1), ctl)) return false;
+        tc_fence_after();
+        const uint32_t kb = sK + (jp & 1) * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDQ, tS + 8u * kk, desc_mnmajor(kb + 2048u * kk), kIdescKMN, (jp > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(BAR_DQDONE));
+        tc_commit(bar(BAR_KEMPTY + (jp & 1)));
+        return true;
+      };
+      int n = -1;
+      if (ok) {
+        n = for_each_chunk(g, tb, list, cnt, [&](int j, int, int, bool) -> bool {
+          const int s = j & 1;
+          const uint32_t ph = (uint32_t)((j >> 1) & 1);
+          if (j > 0 && !dq_step(j - 1)) return false;
+          if (!wait_bounded(bar(BAR_KFULL + s), ph, ctl)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tS, desc_kmajor(sQ + off), desc_kmajor(sK + s * kTileBytes + off), kIdescKK, kk > 0 ? 1u : 0u);
+          }
+          if (!wait_bounded(bar(BAR_VFULL + s), ph, ctl)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tP, desc_kmajor(sDO + off), desc_kmajor(sV + s * kTileBytes + off), kIdescKK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(BAR_SFULL));
+          tc_commit(bar(BAR_VEMPTY + s));
+          return true;
+        });
+      }
+      if (n > 0) dq_step(n - 1);
+      tc_commit(bar(BAR_DRAIN));
+      drain_wait(bar(BAR_DRAIN), 0, kTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------ P, dS and the epilogue
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int64_t row = (int64_t)qrow0 + warp * 32 + lane;
+    const int qoff = (int)(row - (int64_t)qt * g.N);
+    const bool row_ok = row < g.Lq && key_valid(g, qt, qoff);
+    const float L2 = row_ok ? __ldg(lse + bh * g.Lq + row) * 1.4426950408889634f : 0.f;
+    const bool live = row_ok && L2 > -INFINITY;
+    const float Dr = live ? __ldg(Dv + bh * g.Lq + row) : 0.f;
+    const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool full) -> bool {
+      if (!wait_warp(bar(BAR_SFULL), (uint32_t)(j & 1), ctl)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float sv[64], dpv[64];
+        tmem_ld64(tS + lane_off + 64u * half, sv);
+        tmem_ld64(tP + lane_off + 64u * half, dpv);
+        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;   // valid keys of columns 64 half + [0,32), [32,64)
+        if (!full) {
+          vm0 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + lane));
+          vm1 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + 32 + lane));
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * i + e;
+            const bool kv = ((c < 32 ? vm0 >> c : vm1 >> (c - 32)) & 1u) != 0;
+            const float p = (live && kv) ? ex2(sv[c] * scale_log2 - L2) : 0.f;
+            ds[e] = p * (dpv[c] - Dr);
+          }
+          pk[i] = pack_bf16x2(ds[0], ds[1]);
+        }
+        tmem_st32u(tS + lane_off + 32u * half, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(BAR_DSREADY));
+      return true;
+    });
+    // epilogue: dQ * scale in bf16 (pad rows and rows without keys write zeros)
+    bool have = n > 0;
+    if (have) have = wait_warp(bar(BAR_DQDONE), (uint32_t)((n - 1) & 1), ctl);
+    tc_fence_after();
+    const bool write = row < g.Lq && !*abort_flag;
+    const float sc = scale_log2 * 0.69314718055994531f;   // the softmax scale
+    __nv_bfloat16* orow = dq + (bh * g.Lq + row) * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float v[32];
+      if (have) {
+        tmem_ld32(tDQ + lane_off + 32u * q, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (write) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+          const float m = row_ok ? sc : 0.f;
+          uint4 pkv;
+          pkv.x = pack_bf16x2(v[8 * w4 + 0] * m, v[8 * w4 + 1] * m);
+          pkv.y = pack_bf16x2(v[8 * w4 + 2] * m, v[8 * w4 + 3] * m);
+          pkv.z = pack_bf16x2(v[8 * w4 + 4] * m, v[8 * w4 + 5] * m);
+          pkv.w = pack_bf16x2(v[8 * w4 + 6] * m, v[8 * w4 + 7] * m);
+          dst[w4] = pkv;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
+                                       const float* lse, const float* Dv, const int32_t* kv_idx,
+                                       const int32_t* kv_cnt, void* dq, int32_t* status, cudaStream_t s) {
+  const int64_t BH = (int64_t)g.B * g.H;
+  if (BH == 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, g) || !make_map(&mk, k, g) || !make_map(&mv, v, g) || !make_map(&mdo, dO, g))
+    return cudaErrorInvalidValue;
+  static std::atomic<bool> attr_set[64];
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_release);
+  }
+  const int64_t units = BH * (int64_t)g.NQ * (g.N / 128);
+  bwd_dq_tc_kernel<<<(unsigned)units, kThreads, kSmemAlloc, s>>>(mq, mk, mv, mdo, g, make_chunk_tables(g), kv_idx,
+                                                                   kv_cnt, lse, Dv, static_cast<__nv_bfloat16*>(dq),
+                                                                   status, g.scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
+}  // namespace ssta

@@ -93,6 +93,10 @@ cudaError_t launch_attention_f32(const Geom& g, const float* qp, const float* kp
 cudaError_t launch_attention_bwd(const Geom& g, const void* q, const void* k, const void* v, const void* o,
                                  const float* lse, const void* dO, const int32_t* kv_idx, const int32_t* kv_cnt,
                                  void* dq, void* dk, void* dv, void* workspace, cudaStream_t s);
+// bf16, N % 128 == 0: dQ on the tensor cores (Dv = rowsum(dO * O) already computed).
+cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
+                                       const float* lse, const float* Dv, const int32_t* kv_idx,
+                                       const int32_t* kv_cnt, void* dq, int32_t* status, cudaStream_t s);
 cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* kp, const void* vp,
                                      const int32_t* kv_idx, const int32_t* kv_cnt, void* o, float* lse,
                                      int32_t* status, cudaStream_t s);

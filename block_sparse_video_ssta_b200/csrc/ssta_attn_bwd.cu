@@ -14,9 +14,11 @@
 //                         in every query tile's sorted list, ballots, prefix).
 //   bwd_dq_kernel         one warp per query row, walking its tile's kept list
 //                         (fp32; bf16 runs bwd_dq_tc_kernel on the tensor cores).
-//   bwd_dkdv_kernel       one warp per key row, walking the transposed list.
-// The SIMT kernels use fp32 arithmetic, one lane per four channels; for bf16 the
-// dQ products run on the tensor cores, dK and dV do not yet.
+//   bwd_dkdv_kernel       one warp per key row, walking the transposed list
+//                         (fp32; bf16 runs bwd_dkdv_tc_kernel on the tensor cores).
+// The SIMT kernels (fp32 storage) use fp32 arithmetic, one lane per four
+// channels; for bf16 every product runs on the tensor cores
+// (ssta_attn_bwd_tc.cu).
 #include "ssta_internal.h"
 
 #include <cuda_bf16.h>
@@ -222,7 +224,7 @@ bwd_dkdv_kernel(Geom g, const T* __restrict__ qp, const T* __restrict__ kp, cons
 }
 
 template <typename T>
-constexpr bool kTensorCores = false;   // bf16: dQ runs on the tensor cores (ssta_attn_bwd_tc.cu)
+constexpr bool kTensorCores = false;   // bf16: dQ, dK and dV run on the tensor cores (ssta_attn_bwd_tc.cu)
 template <>
 constexpr bool kTensorCores<__nv_bfloat16> = true;
 
@@ -249,8 +251,13 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
     bwd_dq_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, kv_idx, kv_cnt, static_cast<T*>(dq),
                                                    status);
   }
-  bwd_dkdv_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, tidx, tcnt, static_cast<T*>(dk),
-                                                   static_cast<T*>(dv));
+  if (kTensorCores<T> && g.N % 128 == 0) {
+    const cudaError_t e = launch_attention_bwd_dkdv_tc(g, q, k, v, dO, lse, Dv, tidx, tcnt, dk, dv, status, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    bwd_dkdv_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, tidx, tcnt, static_cast<T*>(dk),
+                                                     static_cast<T*>(dv));
+  }
   return cudaGetLastError();
 }
 

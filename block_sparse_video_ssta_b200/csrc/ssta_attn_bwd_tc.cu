@@ -311,4 +311,340 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
   return cudaGetLastError();
 }
 
+// ============================================================================
+// dK and dV on the tensor cores:  dV = P^T dO,  dK = scale * dS^T Q, for one
+// 128-key block, summed over the 128-row query chunks of every query tile that
+// keeps the block's tile (the transposed kept lists).  Warp roles:
+//   warps 0-3  one thread per key row: P^T and dS^T from S^T and dP^T in tensor
+//              memory (the per-query LSE and D come from shared memory);
+//              P^T (bf16) over S^T, dS^T (bf16) over dP^T; epilogue
+//   warp  4    producer: K and V of the block once; per step Q and dO by TMA and
+//              the step's LSE (log2 units, +inf for rows without meaning) and D,
+//              loaded and stored to shared memory by the warp's 32 lanes
+//   warp  5    TMEM allocator and MMA issuer: per step dV, dK of the previous
+//              step (A from tensor memory, B = dO and Q read MN-major), then
+//              S^T = K Q^T and dP^T = V dO^T
+// Tensor memory: S^T | dP^T | dV | dK, 128 columns each.
+// ============================================================================
+namespace {
+
+using namespace wait;
+using namespace tc;
+
+constexpr int kKvThreads = 192;
+constexpr uint32_t kKvOffK = 0;
+constexpr uint32_t kKvOffV = kTileBytes;
+constexpr uint32_t kKvStageBytes = 2 * kTileBytes + 1024;   // Q | dO | L2[128] | D[128]
+constexpr uint32_t kKvOffStage = 2 * kTileBytes;
+constexpr uint32_t kKvOffBar = kKvOffStage + 2 * kKvStageBytes;
+constexpr int kKvNumBars = 10;
+constexpr uint32_t kKvOffMisc = kKvOffBar + kKvNumBars * 8;
+constexpr uint32_t kKvSmemAlloc = kKvOffMisc + 64 + 1024;
+
+enum : int {
+  KB_KV = 0, KB_QFULL = 1, KB_QEMPTY = 3, KB_SFULL = 5, KB_PREADY = 6, KB_DONE = 7, KB_DRAIN = 8
+};
+
+// Calls f(step, t, ch) for every 128-row chunk with a valid row of every query tile
+// in the transposed list, in list order; stops early when f returns false.
+template <typename F>
+__device__ __forceinline__ int for_each_qchunk(const Geom& g, const ChunkTables& tb, const int32_t* tlist, int tcount,
+                                               F&& f) {
+  const int nch = g.N / kChunk;
+  int step = 0;
+  for (int e = 0; e < tcount; ++e) {
+    const int t = __ldg(tlist + e);
+    uint32_t any, full;
+    chunk_bits(g, tb, t, any, full);
+    for (int ch = 0; ch < nch; ++ch) {
+      if (!((any >> ch) & 1u)) continue;
+      if (!f(step, t, ch)) return -1;
+      ++step;
+    }
+  }
+  return step;
+}
+
+__global__ void __launch_bounds__(kKvThreads, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Geom g,
+                   const ChunkTables tb, const int32_t* __restrict__ tidx, const int32_t* __restrict__ tcnt,
+                   const float* __restrict__ lse, const float* __restrict__ Dv, __nv_bfloat16* __restrict__ dk,
+                   __nv_bfloat16* __restrict__ dv, int32_t* __restrict__ status, float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t sK = base + kKvOffK, sV = base + kKvOffV;
+  auto stage = [&](int s) { return base + kKvOffStage + (uint32_t)s * kKvStageBytes; };
+  auto stage_ptr = [&](int s) { return base_ptr + kKvOffStage + (size_t)s * kKvStageBytes; };
+  auto bar = [&](int i) { return base + kKvOffBar + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kKvOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kKvOffMisc + 8);
+  volatile int* bad_list = reinterpret_cast<volatile int*>(base_ptr + kKvOffMisc + 16);
+  const Ctl ctl{abort_flag, status, kTimeoutNs};
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: one 128-key block of a key tile; text key tiles first (longest lists)
+  const int blocks = g.N / 128;
+  const int64_t BH = (int64_t)g.B * g.H;
+  const int64_t text_units = BH * g.n_text * blocks;
+  int64_t u = blockIdx.x;
+  int64_t bh;
+  int kt, blk;
+  if (u < text_units) {
+    bh = u / ((int64_t)g.n_text * blocks);
+    const int rem = (int)(u - bh * g.n_text * blocks);
+    kt = g.NT + rem / blocks;
+    blk = rem % blocks;
+  } else {
+    u -= text_units;
+    bh = u / ((int64_t)g.NT * blocks);
+    const int rem = (int)(u - bh * g.NT * blocks);
+    kt = rem / blocks;
+    blk = rem % blocks;
+  }
+  const int krow0 = kt * g.N + blk * 128;
+  const int64_t trow = bh * g.NQ + kt;
+  int tcount = __ldg(tcnt + trow);
+  if (tcount < 0 || tcount > g.NQ) {
+    if (threadIdx.x == 0) atomicExch(status, (int)SSTA_ERR_DEVICE_BOUNDS);
+    tcount = tcount < 0 ? 0 : g.NQ;
+  }
+  const int32_t* tlist = tidx + trow * g.NQ;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(KB_KV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(KB_QFULL + s), 33);      // the TMA transaction arrival + 32 producer lanes
+      mbar_init(bar(KB_QEMPTY + s), 1);
+    }
+    mbar_init(bar(KB_SFULL), 1);
+    mbar_init(bar(KB_PREADY), 128);
+    mbar_init(bar(KB_DONE), 1);
+    mbar_init(bar(KB_DRAIN), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    *bad_list = 0;
+    for (int e = 0; e < tcount; ++e) {
+      const int t = __ldg(tlist + e);
+      if (t < 0 || t >= g.NQ) { atomicExch(status, (int)SSTA_ERR_DEVICE_BOUNDS); *bad_list = 1; break; }
+    }
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // a bad list entry (recorded above) walks no query chunk at all
+  if (*bad_list) tcount = 0;
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+
+  if (warp == kProducerWarp) {
+    // ---------------------------------------------------------------- producer
+    const int z = (int)bh;
+    if (lane == 0) {
+      mbar_expect_tx(bar(KB_KV), 2 * kTileBytes);
+      for (int b = 0; b < 2; ++b) {
+        tma_load_3d(sK + b * kBox, &tmK, b * 64, krow0, z, bar(KB_KV));
+        tma_load_3d(sV + b * kBox, &tmV, b * 64, krow0, z, bar(KB_KV));
+      }
+    }
+    int issued[2] = {0, 0};
+    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int t, int ch) -> bool {
+      const int s = step & 1;
+      const uint32_t ph = (uint32_t)((step >> 1) & 1);
+      if (!wait_warp(bar(KB_QEMPTY + s), ph ^ 1u, ctl)) return false;
+      const int qrow = t * g.N + ch * kChunk;
+      if (lane == 0) {
+        mbar_expect_tx(bar(KB_QFULL + s), 2 * kTileBytes);
+        for (int b = 0; b < 2; ++b) {
+          tma_load_3d(stage(s) + b * kBox, &tmQ, b * 64, qrow, z, bar(KB_QFULL + s));
+          tma_load_3d(stage(s) + kTileBytes + b * kBox, &tmDO, b * 64, qrow, z, bar(KB_QFULL + s));
+        }
+      }
+      float* l2 = reinterpret_cast<float*>(stage_ptr(s) + 2 * kTileBytes);
+      float* dd = l2 + 128;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        const int64_t row = (int64_t)qrow + c;
+        const bool ok = row < g.Lq && key_valid(g, t, ch * kChunk + c);
+        const float L = ok ? __ldg(lse + bh * g.Lq + row) : -INFINITY;
+        l2[c] = L > -INFINITY ? L * 1.4426950408889634f : INFINITY;   // +inf: the row contributes nothing
+        dd[c] = L > -INFINITY ? __ldg(Dv + bh * g.Lq + row) : 0.f;
+      }
+      mbar_arrive(bar(KB_QFULL + s));
+      ++issued[s];
+      return true;
+    });
+    if (n < 0 && lane == 0) {
+      drain_wait(bar(KB_KV), 0, kTimeoutNs);
+      for (int s = 0; s < 2; ++s)
+        if (issued[s] > 0) drain_wait(bar(KB_QFULL + s), (uint32_t)((issued[s] - 1) & 1), kTimeoutNs);
+    }
+    if (n >= 0 && lane == 0 && tcount == 0) drain_wait(bar(KB_KV), 0, kTimeoutNs);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const bool ok = wait_bounded(bar(KB_KV), 0, ctl);
+      auto grad_step = [&](int sp) -> bool {   // dV, dK of step sp
+        if (!wait_bounded(bar(KB_PREADY), (uint32_t)(sp & 1), ctl)) return false;
+        tc_fence_after();
+        const uint32_t qb = stage(sp & 1), ob = qb + kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDV, tS + 8u * kk, desc_mnmajor(ob + 2048u * kk), kIdescKMN, (sp > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDK, tP + 8u * kk, desc_mnmajor(qb + 2048u * kk), kIdescKMN, (sp > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(KB_DONE));
+        tc_commit(bar(KB_QEMPTY + (sp & 1)));
+        return true;
+      };
+      int n = -1;
+      if (ok) {
+        n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
+          const int s = step & 1;
+          if (step > 0 && !grad_step(step - 1)) return false;
+          if (!wait_bounded(bar(KB_QFULL + s), (uint32_t)((step >> 1) & 1), ctl)) return false;
+          tc_fence_after();
+          const uint32_t qb = stage(s), ob = qb + kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tS, desc_kmajor(sK + off), desc_kmajor(qb + off), kIdescKK, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tP, desc_kmajor(sV + off), desc_kmajor(ob + off), kIdescKK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(KB_SFULL));
+          return true;
+        });
+      }
+      if (n > 0) grad_step(n - 1);
+      tc_commit(bar(KB_DRAIN));
+      drain_wait(bar(KB_DRAIN), 0, kTimeoutNs);
+    }
+  } else {
+    // --------------------------------------------- P^T, dS^T and the epilogue
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int64_t row = (int64_t)krow0 + warp * 32 + lane;
+    const bool key_ok = row < g.Lq && key_valid(g, kt, (int)(row - (int64_t)kt * g.N));
+    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
+      if (!wait_warp(bar(KB_SFULL), (uint32_t)(step & 1), ctl)) return false;
+      // the producer's per-query values of this stage: acquire them from its own barrier
+      if (!wait_warp(bar(KB_QFULL + (step & 1)), (uint32_t)((step >> 1) & 1), ctl)) return false;
+      tc_fence_after();
+      const float* l2 = reinterpret_cast<const float*>(stage_ptr(step & 1) + 2 * kTileBytes);
+      const float* dd = l2 + 128;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float sv[64], dpv[64];
+        tmem_ld64(tS + lane_off + 64u * half, sv);
+        tmem_ld64(tP + lane_off + 64u * half, dpv);
+        uint32_t pkp[32], pks[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 L = reinterpret_cast<const float4*>(l2 + 64 * half)[i];
+          const float4 Dq = reinterpret_cast<const float4*>(dd + 64 * half)[i];
+          const float Ls[4] = {L.x, L.y, L.z, L.w}, Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
+          float p[4], ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool live = Ls[e] < INFINITY;   // +inf marks a query row without meaning
+            p[e] = live ? ex2(sv[4 * i + e] * scale_log2 - Ls[e]) : 0.f;
+            ds[e] = live ? p[e] * (dpv[4 * i + e] - Ds[e]) : 0.f;
+          }
+          pkp[2 * i] = pack_bf16x2(p[0], p[1]);
+          pkp[2 * i + 1] = pack_bf16x2(p[2], p[3]);
+          pks[2 * i] = pack_bf16x2(ds[0], ds[1]);
+          pks[2 * i + 1] = pack_bf16x2(ds[2], ds[3]);
+        }
+        tmem_st32u(tS + lane_off + 32u * half, pkp);
+        tmem_st32u(tP + lane_off + 32u * half, pks);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(KB_PREADY));
+      return true;
+    });
+    bool have = n > 0;
+    if (have) have = wait_warp(bar(KB_DONE), (uint32_t)((n - 1) & 1), ctl);
+    tc_fence_after();
+    const bool write = row < g.Lq && !*abort_flag;
+    const float sc = scale_log2 * 0.69314718055994531f;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      __nv_bfloat16* orow = (which ? dk : dv) + (bh * g.Lq + row) * 128;
+      const float m = key_ok ? (which ? sc : 1.0f) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        if (have) {
+          tmem_ld32((which ? tDK : tDV) + lane_off + 32u * q, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        if (write) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
+#pragma unroll
+          for (int w4 = 0; w4 < 4; ++w4) {
+            uint4 pkv;
+            pkv.x = pack_bf16x2(v[8 * w4 + 0] * m, v[8 * w4 + 1] * m);
+            pkv.y = pack_bf16x2(v[8 * w4 + 2] * m, v[8 * w4 + 3] * m);
+            pkv.z = pack_bf16x2(v[8 * w4 + 4] * m, v[8 * w4 + 5] * m);
+            pkv.w = pack_bf16x2(v[8 * w4 + 6] * m, v[8 * w4 + 7] * m);
+            dst[w4] = pkv;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention_bwd_dkdv_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
+                                         const float* lse, const float* Dv, const int32_t* tidx,
+                                         const int32_t* tcnt, void* dk, void* dv, int32_t* status, cudaStream_t s) {
+  const int64_t BH = (int64_t)g.B * g.H;
+  if (BH == 0) return cudaSuccess;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, g) || !make_map(&mk, k, g) || !make_map(&mv, v, g) || !make_map(&mdo, dO, g))
+    return cudaErrorInvalidValue;
+  static std::atomic<bool> attr_set[64];
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kKvSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_release);
+  }
+  const int64_t units = BH * (int64_t)g.NQ * (g.N / 128);
+  bwd_dkdv_tc_kernel<<<(unsigned)units, kKvThreads, kKvSmemAlloc, s>>>(
+      mq, mk, mv, mdo, g, make_chunk_tables(g), tidx, tcnt, lse, Dv, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv), status, g.scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
 }  // namespace ssta

@@ -97,6 +97,10 @@ cudaError_t launch_attention_bwd(const Geom& g, const void* q, const void* k, co
 cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
                                        const float* lse, const float* Dv, const int32_t* kv_idx,
                                        const int32_t* kv_cnt, void* dq, int32_t* status, cudaStream_t s);
+// bf16, N % 128 == 0: dK and dV on the tensor cores (tidx/tcnt: the transposed lists).
+cudaError_t launch_attention_bwd_dkdv_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
+                                         const float* lse, const float* Dv, const int32_t* tidx,
+                                         const int32_t* tcnt, void* dk, void* dv, int32_t* status, cudaStream_t s);
 cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* kp, const void* vp,
                                      const int32_t* kv_idx, const int32_t* kv_cnt, void* o, float* lse,
                                      int32_t* status, cudaStream_t s);

@@ -198,7 +198,9 @@ ssta_status ssta_attention_fwd(const ssta_desc* desc, const void* q_packed, cons
  *   required), dq/dk/dv_packed [B,H,Lq,D] (written in full), all of `dtype`;
  *   workspace >= info.bwd_workspace_bytes (status word, per-row D, and for every key
  *   tile the list of query tiles keeping it).
- * SIMT kernels (fp32 arithmetic); the products are not on the tensor cores.
+ * bf16 with N % 128 == 0: tcgen05 tensor-core kernels (one for dQ over each query
+ * tile's kept list, one for dK and dV over the query tiles keeping each key tile);
+ * fp32 (or other N): SIMT kernels with fp32 arithmetic.
  */
 ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, const void* k_packed,
                                const void* v_packed, const void* o_packed, const float* lse,

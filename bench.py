@@ -550,7 +550,8 @@ def run_backward(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "pass": "backward", "grid": [w.T, w.Y, w.X], "heads": w.H,
                    "mask": {"score": w.score_mode, "combine": w.combine, "window": w.window_mode},
-                   "kernels": "SIMT (fp32 arithmetic), not tensor cores"},
+                   "kernels": ("tcgen05 tensor cores (dQ and dK/dV kernels)" if w.dtype == "bf16" and (w.tX * w.tY * w.tT) % 128 == 0
+                               else "SIMT (fp32 storage)")},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
                      "peak_source": f"{src} bf16_tflops_sustained", "traffic": None},
         "gpu_launches": 4 * args.steps, "clocks": clk.summary(),

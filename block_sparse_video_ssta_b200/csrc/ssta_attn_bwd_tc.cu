@@ -6,16 +6,18 @@
 //
 // One CTA owns 128 query rows of one query tile and walks the tile's kept list
 // in 128-key chunks.  Warp roles:
-//   warps 0-3  one thread per query row: P and dS from S and dP in tensor
-//              memory; dS (bf16) is written over S; epilogue dQ * scale
-//   warp  4    TMA producer: Q and dO once, then K and V chunks (2-stage rings)
-//   warp  5    TMEM allocator and tcgen05.mma issuer
-// Tensor memory: S (fp32, 128 columns; dS as bf16 over its first 64), dP
-// (128 columns), dQ accumulator (128 columns).
-// Per chunk j the MMA warp issues dQ += dS(j-1) K(j-1) (A = dS from tensor
-// memory, B = K in shared memory read MN-major), then S(j) = Q K(j)^T and
-// dP(j) = dO V(j)^T (both from shared memory).  The pipe executes in order, so
-// S(j) overwrites dS(j-1) only after dQ has read it.
+//   warps 0-7  elementwise: warp w serves query rows 32 (w mod 4) .. +31 and key
+//              columns 64 (w / 4) .. +63 of each chunk: P and dS from S and dP in
+//              tensor memory, dS (bf16) into shared memory; epilogue dQ * scale
+//   warp  8    TMA producer: Q and dO once, then K and V chunks (2-stage rings)
+//   warp  9    TMEM allocator and tcgen05.mma issuer
+// Tensor memory: S (fp32, 128 columns), dP (128 columns), dQ accumulator (128).
+// Shared memory: Q, dO, the K and V rings and dS (K-major, 128-byte swizzle).
+// Per chunk j the MMA warp issues S(j) = Q K(j)^T and dP(j) = dO V(j)^T as soon
+// as the elementwise warps have loaded S(j-1) and dP(j-1) into registers, then
+// dQ += dS(j-1) K(j-1) (A = dS from shared memory, B = K read MN-major) once
+// dS(j-1) is written: the next chunk's S and dP run during this chunk's
+// exponentials.  dS is overwritten only after the previous dQ product finished.
 // Every wait is bounded (ssta_wait.cuh), as in the forward kernel.
 #include "ssta_tc_common.cuh"
 
@@ -25,27 +27,32 @@ namespace {
 using namespace wait;
 using namespace tc;
 
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 1500000000ull;
+
+// dQ kernel: 8 elementwise warps (two per TMEM lane group, 64 key columns each),
+// the producer and the MMA issuer.
+constexpr int kDqThreads = 320;
+constexpr int kDqProducerWarp = 8;
+constexpr int kDqMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffDO = kOffQ + kTileBytes;
 constexpr uint32_t kOffK = kOffDO + kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffDS = kOffV + kStages * kTileBytes;   // dS (bf16), K-major, 128-byte swizzle
+constexpr uint32_t kOffBar = kOffDS + kTileBytes;
 constexpr int kNumBars = 14;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemAlloc = kOffMisc + 64 + 1024;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kTimeoutNs = 1500000000ull;
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 
 enum : int {
   BAR_Q = 0, BAR_KFULL = 1, BAR_KEMPTY = 3, BAR_VFULL = 5, BAR_VEMPTY = 7,
-  BAR_SFULL = 9, BAR_DSREADY = 10, BAR_DQDONE = 11, BAR_DRAIN = 12
+  BAR_SFULL = 9, BAR_SFREE = 10, BAR_DSREADY = 11, BAR_DQDONE = 12, BAR_DRAIN = 13
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Geom g,
                  const ChunkTables tb, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
@@ -55,7 +62,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t sQ = base + kOffQ, sDO = base + kOffDO, sK = base + kOffK, sV = base + kOffV;
+  const uint32_t sQ = base + kOffQ, sDO = base + kOffDO, sK = base + kOffK, sV = base + kOffV, sDS = base + kOffDS;
   auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffMisc + 8);
@@ -100,7 +107,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(bar(BAR_VEMPTY + s), 1);
     }
     mbar_init(bar(BAR_SFULL), 1);
-    mbar_init(bar(BAR_DSREADY), 128);
+    mbar_init(bar(BAR_SFREE), 256);
+    mbar_init(bar(BAR_DSREADY), 256);
     mbar_init(bar(BAR_DQDONE), 1);
     mbar_init(bar(BAR_DRAIN), 1);
     *abort_flag = 0;
@@ -110,7 +118,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (t < 0 || t >= g.NQ) { atomicExch(status, (int)SSTA_ERR_DEVICE_BOUNDS); break; }
     }
   }
-  if (warp == kMmaWarp) {
+  if (warp == kDqMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
@@ -122,7 +130,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tP = tmem + 128, tDQ = tmem + 256;
 
-  if (warp == kProducerWarp) {
+  if (warp == kDqProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int z = (int)bh;
@@ -156,18 +164,23 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kDqMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
+    // Per chunk j: S(j) = Q K(j)^T and dP(j) = dO V(j)^T as soon as the elementwise
+    // warps have loaded S(j-1) and dP(j-1), then dQ += dS(j-1) K(j-1) once dS(j-1) is
+    // in shared memory, so S and dP of the next chunk run during this chunk's exponentials.
     if (lane == 0) {
       const bool ok = wait_bounded(bar(BAR_Q), 0, ctl);
-      // dQ += dS(jp) K(jp): A = dS (bf16, columns 0..63 of S), B = K stage read MN-major
+      // dQ += dS(jp) K(jp): A = dS (K-major in shared memory), B = K stage read MN-major
       auto dq_step = [&](int jp) -> bool {
         if (!wait_bounded(bar(BAR_DSREADY), (uint32_t)(jp & 1), ctl)) return false;
         tc_fence_after();
         const uint32_t kb = sK + (jp & 1) * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDQ, tS + 8u * kk, desc_mnmajor(kb + 2048u * kk), kIdescKMN, (jp > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+          mma_ss(tDQ, desc_kmajor(sDS + off), desc_mnmajor(kb + 2048u * kk), kIdescKMN, (jp > 0 || kk > 0) ? 1u : 0u);
+        }
         tc_commit(bar(BAR_DQDONE));
         tc_commit(bar(BAR_KEMPTY + (jp & 1)));
         return true;
@@ -177,7 +190,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         n = for_each_chunk(g, tb, list, cnt, [&](int j, int, int, bool) -> bool {
           const int s = j & 1;
           const uint32_t ph = (uint32_t)((j >> 1) & 1);
-          if (j > 0 && !dq_step(j - 1)) return false;
+          if (j > 0) {
+            if (!wait_bounded(bar(BAR_SFREE), (uint32_t)((j - 1) & 1), ctl)) return false;
+            tc_fence_after();
+          }
           if (!wait_bounded(bar(BAR_KFULL + s), ph, ctl)) return false;
           tc_fence_after();
 #pragma unroll
@@ -194,7 +210,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
           tc_commit(bar(BAR_SFULL));
           tc_commit(bar(BAR_VEMPTY + s));
-          return true;
+          return j == 0 ? true : dq_step(j - 1);
         });
       }
       if (n > 0) dq_step(n - 1);
@@ -203,58 +219,67 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else {
     // ------------------------------------------------ P, dS and the epilogue
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int64_t row = (int64_t)qrow0 + warp * 32 + lane;
+    // warp w: TMEM lanes 32 (w mod 4) .. +31 (its query rows), key columns 64 (w / 4) .. +63
+    const int grp = warp & 3, half = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
+    const int r = grp * 32 + lane;   // row within the block
+    const int64_t row = (int64_t)qrow0 + r;
     const int qoff = (int)(row - (int64_t)qt * g.N);
     const bool row_ok = row < g.Lq && key_valid(g, qt, qoff);
     const float L2 = row_ok ? __ldg(lse + bh * g.Lq + row) * 1.4426950408889634f : 0.f;
     const bool live = row_ok && L2 > -INFINITY;
     const float Dr = live ? __ldg(Dv + bh * g.Lq + row) : 0.f;
+    uint8_t* ds_row = base_ptr + kOffDS + half * kBox + r * 128;   // this thread's 64 keys: one box row
     const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool full) -> bool {
       if (!wait_warp(bar(BAR_SFULL), (uint32_t)(j & 1), ctl)) return false;
       tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float sv[64], dpv[64];
-        tmem_ld64(tS + lane_off + 64u * half, sv);
-        tmem_ld64(tP + lane_off + 64u * half, dpv);
-        uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;   // valid keys of columns 64 half + [0,32), [32,64)
-        if (!full) {
-          vm0 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + lane));
-          vm1 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + 32 + lane));
-        }
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * i + e;
-            const bool kv = ((c < 32 ? vm0 >> c : vm1 >> (c - 32)) & 1u) != 0;
-            const float p = (live && kv) ? ex2(sv[c] * scale_log2 - L2) : 0.f;
-            ds[e] = p * (dpv[c] - Dr);
-          }
-          pk[i] = pack_bf16x2(ds[0], ds[1]);
-        }
-        tmem_st32u(tS + lane_off + 32u * half, pk);
-      }
-      tmem_wait_st();
+      float sv[64], dpv[64];
+      tmem_ld64(tS + lane_off + 64u * half, sv);
+      tmem_ld64(tP + lane_off + 64u * half, dpv);
       tc_fence_before();
+      mbar_arrive(bar(BAR_SFREE));   // S and dP of this chunk are in registers
+      uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;   // valid keys of columns [0,32), [32,64) of this half
+      if (!full) {
+        vm0 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + lane));
+        vm1 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + 32 + lane));
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 2 * i + e;
+          const bool kv = ((c < 32 ? vm0 >> c : vm1 >> (c - 32)) & 1u) != 0;
+          const float p = (live && kv) ? ex2(sv[c] * scale_log2 - L2) : 0.f;
+          ds[e] = p * (dpv[c] - Dr);
+        }
+        pk[i] = pack_bf16x2(ds[0], ds[1]);
+      }
+      // dQ(j-1) reads dS from shared memory: it must have finished before dS is overwritten
+      if (j > 0 && !wait_warp(bar(BAR_DQDONE), (uint32_t)((j - 1) & 1), ctl)) return false;
+      // 16-byte chunk c of the row (keys 8c..8c+7 of this half) at position c ^ (r mod 8)
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
       mbar_arrive(bar(BAR_DSREADY));
       return true;
     });
-    // epilogue: dQ * scale in bf16 (pad rows and rows without keys write zeros)
+    // epilogue: dQ * scale in bf16 (pad rows and rows without keys write zeros); warp w
+    // writes channels 64 (w / 4) .. +63 of its rows
     bool have = n > 0;
     if (have) have = wait_warp(bar(BAR_DQDONE), (uint32_t)((n - 1) & 1), ctl);
     tc_fence_after();
     const bool write = row < g.Lq && !*abort_flag;
     const float sc = scale_log2 * 0.69314718055994531f;   // the softmax scale
-    __nv_bfloat16* orow = dq + (bh * g.Lq + row) * 128;
+    __nv_bfloat16* orow = dq + (bh * g.Lq + row) * 128 + 64 * half;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
       float v[32];
       if (have) {
-        tmem_ld32(tDQ + lane_off + 32u * q, v);
+        tmem_ld32(tDQ + lane_off + 64u * half + 32u * q, v);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0.f;
@@ -277,7 +302,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kDqMmaWarp) {
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
@@ -305,7 +330,7 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
     attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t units = BH * (int64_t)g.NQ * (g.N / 128);
-  bwd_dq_tc_kernel<<<(unsigned)units, kThreads, kSmemAlloc, s>>>(mq, mk, mv, mdo, g, make_chunk_tables(g), kv_idx,
+  bwd_dq_tc_kernel<<<(unsigned)units, kDqThreads, kSmemAlloc, s>>>(mq, mk, mv, mdo, g, make_chunk_tables(g), kv_idx,
                                                                    kv_cnt, lse, Dv, static_cast<__nv_bfloat16*>(dq),
                                                                    status, g.scale * 1.4426950408889634f);
   return cudaGetLastError();
@@ -315,13 +340,15 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
 // dK and dV on the tensor cores:  dV = P^T dO,  dK = scale * dS^T Q, for one
 // 128-key block, summed over the 128-row query chunks of every query tile that
 // keeps the block's tile (the transposed kept lists).  Warp roles:
-//   warps 0-3  one thread per key row: P^T and dS^T from S^T and dP^T in tensor
-//              memory (the per-query LSE and D come from shared memory);
-//              P^T (bf16) over S^T, dS^T (bf16) over dP^T; epilogue
-//   warp  4    producer: K and V of the block once; per step Q and dO by TMA and
+//   warps 0-7  elementwise: warp w serves key rows 32 (w mod 4) .. +31 and query
+//              columns 64 (w / 4) .. +63 of each step: P^T and dS^T from S^T and
+//              dP^T in tensor memory (the per-query LSE and D come from shared
+//              memory); P^T (bf16) over S^T, dS^T (bf16) over dP^T; epilogue
+//              (the warps of query half 0 write dV, those of half 1 dK)
+//   warp  8    producer: K and V of the block once; per step Q and dO by TMA and
 //              the step's LSE (log2 units, +inf for rows without meaning) and D,
 //              loaded and stored to shared memory by the warp's 32 lanes
-//   warp  5    TMEM allocator and MMA issuer: per step dV, dK of the previous
+//   warp  9    TMEM allocator and MMA issuer: per step dV, dK of the previous
 //              step (A from tensor memory, B = dO and Q read MN-major), then
 //              S^T = K Q^T and dP^T = V dO^T
 // Tensor memory: S^T | dP^T | dV | dK, 128 columns each.
@@ -331,7 +358,9 @@ namespace {
 using namespace wait;
 using namespace tc;
 
-constexpr int kKvThreads = 192;
+constexpr int kKvThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kKvOffK = 0;
 constexpr uint32_t kKvOffV = kTileBytes;
 constexpr uint32_t kKvStageBytes = 2 * kTileBytes + 1024;   // Q | dO | L2[128] | D[128]
@@ -421,7 +450,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(bar(KB_QEMPTY + s), 1);
     }
     mbar_init(bar(KB_SFULL), 1);
-    mbar_init(bar(KB_PREADY), 128);
+    mbar_init(bar(KB_PREADY), 256);
     mbar_init(bar(KB_DONE), 1);
     mbar_init(bar(KB_DRAIN), 1);
     *abort_flag = 0;
@@ -536,8 +565,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else {
     // --------------------------------------------- P^T, dS^T and the epilogue
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int64_t row = (int64_t)krow0 + warp * 32 + lane;
+    // warp w: TMEM lanes 32 (w mod 4) .. +31 (its key rows), query columns 64 (w / 4) .. +63
+    const int grp = warp & 3, half = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
+    const int64_t row = (int64_t)krow0 + grp * 32 + lane;
     const bool key_ok = row < g.Lq && key_valid(g, kt, (int)(row - (int64_t)kt * g.N));
     const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
       if (!wait_warp(bar(KB_SFULL), (uint32_t)(step & 1), ctl)) return false;
@@ -546,66 +577,62 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_after();
       const float* l2 = reinterpret_cast<const float*>(stage_ptr(step & 1) + 2 * kTileBytes);
       const float* dd = l2 + 128;
+      float sv[64], dpv[64];
+      tmem_ld64(tS + lane_off + 64u * half, sv);
+      tmem_ld64(tP + lane_off + 64u * half, dpv);
+      uint32_t pkp[32], pks[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float sv[64], dpv[64];
-        tmem_ld64(tS + lane_off + 64u * half, sv);
-        tmem_ld64(tP + lane_off + 64u * half, dpv);
-        uint32_t pkp[32], pks[32];
+      for (int i = 0; i < 16; ++i) {
+        const float4 L = reinterpret_cast<const float4*>(l2 + 64 * half)[i];
+        const float4 Dq = reinterpret_cast<const float4*>(dd + 64 * half)[i];
+        const float Ls[4] = {L.x, L.y, L.z, L.w}, Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
+        float p[4], ds[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float4 L = reinterpret_cast<const float4*>(l2 + 64 * half)[i];
-          const float4 Dq = reinterpret_cast<const float4*>(dd + 64 * half)[i];
-          const float Ls[4] = {L.x, L.y, L.z, L.w}, Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
-          float p[4], ds[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const bool live = Ls[e] < INFINITY;   // +inf marks a query row without meaning
-            p[e] = live ? ex2(sv[4 * i + e] * scale_log2 - Ls[e]) : 0.f;
-            ds[e] = live ? p[e] * (dpv[4 * i + e] - Ds[e]) : 0.f;
-          }
-          pkp[2 * i] = pack_bf16x2(p[0], p[1]);
-          pkp[2 * i + 1] = pack_bf16x2(p[2], p[3]);
-          pks[2 * i] = pack_bf16x2(ds[0], ds[1]);
-          pks[2 * i + 1] = pack_bf16x2(ds[2], ds[3]);
+        for (int e = 0; e < 4; ++e) {
+          const bool live = Ls[e] < INFINITY;   // +inf marks a query row without meaning
+          p[e] = live ? ex2(sv[4 * i + e] * scale_log2 - Ls[e]) : 0.f;
+          ds[e] = live ? p[e] * (dpv[4 * i + e] - Ds[e]) : 0.f;
         }
-        tmem_st32u(tS + lane_off + 32u * half, pkp);
-        tmem_st32u(tP + lane_off + 32u * half, pks);
+        pkp[2 * i] = pack_bf16x2(p[0], p[1]);
+        pkp[2 * i + 1] = pack_bf16x2(p[2], p[3]);
+        pks[2 * i] = pack_bf16x2(ds[0], ds[1]);
+        pks[2 * i + 1] = pack_bf16x2(ds[2], ds[3]);
       }
+      tmem_st32u(tS + lane_off + 32u * half, pkp);
+      tmem_st32u(tP + lane_off + 32u * half, pks);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(KB_PREADY));
       return true;
     });
+    // epilogue: the warps of column half 0 write dV, those of half 1 write dK
     bool have = n > 0;
     if (have) have = wait_warp(bar(KB_DONE), (uint32_t)((n - 1) & 1), ctl);
     tc_fence_after();
     const bool write = row < g.Lq && !*abort_flag;
     const float sc = scale_log2 * 0.69314718055994531f;
+    const int which = half;
+    __nv_bfloat16* orow = (which ? dk : dv) + (bh * g.Lq + row) * 128;
+    const float m = key_ok ? (which ? sc : 1.0f) : 0.f;
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      __nv_bfloat16* orow = (which ? dk : dv) + (bh * g.Lq + row) * 128;
-      const float m = key_ok ? (which ? sc : 1.0f) : 0.f;
+    for (int q = 0; q < 4; ++q) {
+      float v[32];
+      if (have) {
+        tmem_ld32((which ? tDK : tDV) + lane_off + 32u * q, v);
+      } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        if (have) {
-          tmem_ld32((which ? tDK : tDV) + lane_off + 32u * q, v);
-        } else {
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (write) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        }
-        if (write) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
-#pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) {
-            uint4 pkv;
-            pkv.x = pack_bf16x2(v[8 * w4 + 0] * m, v[8 * w4 + 1] * m);
-            pkv.y = pack_bf16x2(v[8 * w4 + 2] * m, v[8 * w4 + 3] * m);
-            pkv.z = pack_bf16x2(v[8 * w4 + 4] * m, v[8 * w4 + 5] * m);
-            pkv.w = pack_bf16x2(v[8 * w4 + 6] * m, v[8 * w4 + 7] * m);
-            dst[w4] = pkv;
-          }
+        for (int w4 = 0; w4 < 4; ++w4) {
+          uint4 pkv;
+          pkv.x = pack_bf16x2(v[8 * w4 + 0] * m, v[8 * w4 + 1] * m);
+          pkv.y = pack_bf16x2(v[8 * w4 + 2] * m, v[8 * w4 + 3] * m);
+          pkv.z = pack_bf16x2(v[8 * w4 + 4] * m, v[8 * w4 + 5] * m);
+          pkv.w = pack_bf16x2(v[8 * w4 + 6] * m, v[8 * w4 + 7] * m);
+          dst[w4] = pkv;
         }
       }
     }

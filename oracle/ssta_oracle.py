@@ -327,14 +327,19 @@ def attention(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, kept: np.ndarra
 
 
 def attention_bwd(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, dOp: np.ndarray, kept: np.ndarray,
-                  scale: float | None = None):
+                  scale: float | None = None, q_tiles=None, key_tiles=None):
     """Gradients of Step 4's block-sparse attention, in float64: for every valid
     query row of query tile i and the valid keys of its kept tiles, with
     P = softmax(q k^T * scale) (recomputed), O = P v, D = rowsum(dO * O):
     dS = P * (dO v^T - D), dQ = scale * dS k, dK += scale * dS^T q, dV += P^T dO.
     Pad query rows take no part (their dQ is 0); pad keys get dK = dV = 0; a query
     tile with no kept key contributes nothing.  Returns (dQ, dK, dV), each
-    [B,H,Lq,D] on the packed layout."""
+    [B,H,Lq,D] on the packed layout.
+
+    ``q_tiles`` / ``key_tiles`` (default: all) restrict the result to the dQ rows
+    of those query tiles and the dK, dV rows of those key tiles: only the query
+    tiles in ``q_tiles`` or keeping one of ``key_tiles`` are visited, and every
+    other row is NaN."""
     g = geometry(d)
     scale = 1.0 / math.sqrt(g.D) if not scale else scale
     B, H = qp.shape[:2]
@@ -342,6 +347,8 @@ def attention_bwd(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, dOp: np.nda
     dQ = np.zeros((B, H, g.Lq, g.D))
     dK = np.zeros((B, H, g.Lq, g.D))
     dV = np.zeros((B, H, g.Lq, g.D))
+    qsel = np.ones(g.NQ, dtype=bool) if q_tiles is None else np.isin(np.arange(g.NQ), q_tiles)
+    ksel = np.ones(g.NQ, dtype=bool) if key_tiles is None else np.isin(np.arange(g.NQ), key_tiles)
     for b in range(B):
         for h in range(H):
             q = qp[b, h].astype(np.float64)
@@ -349,6 +356,8 @@ def attention_bwd(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, dOp: np.nda
             v = vp[b, h].astype(np.float64)
             do = dOp[b, h].astype(np.float64)
             for i in range(g.NQ):
+                if not (qsel[i] or (kept[b, h, i] & ksel).any()):
+                    continue
                 r0, r1 = i * g.N, min((i + 1) * g.N, g.Lq)
                 rows = np.arange(r0, r1)[valid[r0:r1]]
                 cols = [np.arange(j * g.N, min((j + 1) * g.N, g.Lq)) for j in np.nonzero(kept[b, h, i])[0]]
@@ -365,6 +374,10 @@ def attention_bwd(d, qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, dOp: np.nda
                 dQ[b, h, rows] = scale * ds @ k[keys]
                 np.add.at(dK[b, h], keys, scale * ds.T @ q[rows])
                 np.add.at(dV[b, h], keys, p.T @ do[rows])
+    tile_of_row = np.arange(g.Lq) // g.N
+    dQ[:, :, ~qsel[tile_of_row]] = np.nan
+    dK[:, :, ~ksel[tile_of_row]] = np.nan
+    dV[:, :, ~ksel[tile_of_row]] = np.nan
     return dQ, dK, dV
 
 

@@ -609,3 +609,28 @@ def test_backward_empty_rows_contribute_nothing():
     g, arrs, r, kept, dO_r, dO_t, dOp, (dQ, dK, dV) = _bwd_case(d, 13, kept_fn)
     assert not kept.any()
     assert not dQ.any() and not dK.any() and not dV.any()
+
+
+def test_backward_restricted_tiles_equal_autograd():
+    """attention_bwd restricted to some dQ tiles and some dK/dV tiles (the form the
+    full-size sampled GPU test uses) gives autograd's values on those rows, NaN elsewhere."""
+    d = with_overrides(_desc(T=4, Y=8, X=6, tT=2, tY=4, tX=3, L_text=37, H=2, D=8), recipe="tile_offset")
+    g = oracle.geometry(d)
+    x = si.make_inputs(d, 13)
+    arrs, r = _run_oracle(d, x)
+    rng = np.random.default_rng(9)
+    kept = rng.random((d.B, d.H, g.NQ, g.NQ)) < 0.4
+    kept[:, :, np.arange(g.NQ), np.arange(g.NQ)] = True
+    dO_r = rng.standard_normal((d.B, d.H, d.T, d.Y, d.X, d.D))
+    dO_t = rng.standard_normal((d.B, d.H, d.L_text, d.D))
+    dOp = oracle.tile_reorder(d, dO_r, dO_t)
+    q_tiles, key_tiles = [0, g.NT - 1, g.NQ - 1], [1, g.NT - 1]
+    got = oracle.attention_bwd(d, r["qp"], r["kp"], r["vp"], dOp, kept, q_tiles=q_tiles, key_tiles=key_tiles)
+    ref = _sdpa_grads(d, arrs, dO_r, dO_t, _token_mask_from_tile_mask(d, kept))
+    tile_of_row = np.arange(g.Lq) // g.N
+    for t, want, sel in zip(got, ref, (q_tiles, key_tiles, key_tiles)):
+        rows = np.isin(tile_of_row, sel)
+        assert np.all(np.isfinite(t[:, :, rows])) and np.all(np.isnan(t[:, :, ~rows]))
+        ras = _to_raster(d, np.where(np.isnan(t), 0.0, t))
+        mask = _to_raster(d, np.broadcast_to(rows[None, None, :, None], t.shape).astype(np.float64)) > 0
+        np.testing.assert_allclose(ras[mask], want[mask], rtol=0, atol=1e-11)

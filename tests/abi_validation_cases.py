@@ -81,6 +81,15 @@ cases.append(("attn_no_workspace", attn(d, ws=None)))
 cases.append(("attn_small_workspace", attn(d, wsb=64)))
 cases.append(("attn_null_q", attn(d, q=None)))
 cases.append(("attn_misaligned_o", attn(d, o=P(A + 2))))
+bwd = lambda dd, ws=P(A), wsb=1 << 30, do=P(A), dk=P(A): call(
+    "ssta_attention_bwd", ctypes.byref(dd), P(A), P(A), P(A), P(A), P(A), do, P(A), P(A), P(A), dk, P(A), ws,
+    ctypes.c_size_t(wsb), None)
+cases.append(("bwd_no_workspace", bwd(d, ws=None)))
+cases.append(("bwd_small_workspace", bwd(d, wsb=64)))
+cases.append(("bwd_ws_misaligned", bwd(d, ws=P(A + 16))))
+cases.append(("bwd_null_do", bwd(d, do=None)))
+cases.append(("bwd_misaligned_dk", bwd(d, dk=P(A + 8))))
+cases.append(("bwd_bad_desc", bwd(desc(topk=-1))))
 cases.append(("read_status_null", call("ssta_read_device_status", None, None, None)))
 lib.ssta_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                            ctypes.c_void_p]

@@ -119,6 +119,7 @@ ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, cons
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
+  if (g.dtype == SSTA_BF16 && g.N % 128 != 0) return SSTA_ERR_UNSUPPORTED;
   const BwdWorkspace ws = bwd_workspace_layout(g);
   if (workspace == nullptr || workspace_bytes < ws.total) return SSTA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return SSTA_ERR_ALIGNMENT;

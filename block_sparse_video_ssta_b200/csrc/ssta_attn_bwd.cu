@@ -244,17 +244,14 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
   const T* tO = static_cast<const T*>(dO);
   bwd_rowdot_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, static_cast<const T*>(o), tO, Dv);
   bwd_transpose_kernel<<<tb, kBwdWarps * 32, 0, s>>>(g, kv_idx, kv_cnt, tidx, tcnt, status);
-  if (kTensorCores<T> && g.N % 128 == 0) {
-    const cudaError_t e = launch_attention_bwd_dq_tc(g, q, k, v, dO, lse, Dv, kv_idx, kv_cnt, dq, status, s);
+  if constexpr (kTensorCores<T>) {   // bf16: the API guarantees N % 128 == 0
+    cudaError_t e = launch_attention_bwd_dq_tc(g, q, k, v, dO, lse, Dv, kv_idx, kv_cnt, dq, status, s);
+    if (e != cudaSuccess) return e;
+    e = launch_attention_bwd_dkdv_tc(g, q, k, v, dO, lse, Dv, tidx, tcnt, dk, dv, status, s);
     if (e != cudaSuccess) return e;
   } else {
     bwd_dq_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, kv_idx, kv_cnt, static_cast<T*>(dq),
                                                    status);
-  }
-  if (kTensorCores<T> && g.N % 128 == 0) {
-    const cudaError_t e = launch_attention_bwd_dkdv_tc(g, q, k, v, dO, lse, Dv, tidx, tcnt, dk, dv, status, s);
-    if (e != cudaSuccess) return e;
-  } else {
     bwd_dkdv_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, tidx, tcnt, static_cast<T*>(dk),
                                                      static_cast<T*>(dv));
   }

@@ -198,9 +198,12 @@ ssta_status ssta_attention_fwd(const ssta_desc* desc, const void* q_packed, cons
  *   required), dq/dk/dv_packed [B,H,Lq,D] (written in full), all of `dtype`;
  *   workspace >= info.bwd_workspace_bytes (status word, per-row D, and for every key
  *   tile the list of query tiles keeping it).
- * bf16 with N % 128 == 0: tcgen05 tensor-core kernels (one for dQ over each query
- * tile's kept list, one for dK and dV over the query tiles keeping each key tile);
- * fp32 (or other N): SIMT kernels with fp32 arithmetic.
+ * bf16 (N % 128 == 0 required, as for ssta_attention_fwd): tcgen05 tensor-core
+ * kernels, one for dQ over each query tile's kept list, one for dK and dV over the
+ * query tiles keeping each key tile.  fp32: SIMT kernels with fp32 arithmetic.
+ * Returns SSTA_ERR_UNSUPPORTED for bf16 with N % 128 != 0, SSTA_ERR_WORKSPACE for a
+ * missing or short workspace, SSTA_ERR_ALIGNMENT for a workspace not 256-byte aligned
+ * or a tensor not 16-byte aligned, SSTA_ERR_INVALID_ARG for a NULL tensor.
  */
 ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, const void* k_packed,
                                const void* v_packed, const void* o_packed, const float* lse,

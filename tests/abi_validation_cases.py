@@ -90,6 +90,7 @@ cases.append(("bwd_ws_misaligned", bwd(d, ws=P(A + 16))))
 cases.append(("bwd_null_do", bwd(d, do=None)))
 cases.append(("bwd_misaligned_dk", bwd(d, dk=P(A + 8))))
 cases.append(("bwd_bad_desc", bwd(desc(topk=-1))))
+cases.append(("bwd_bf16_tile_not_128", bwd(desc(dtype=S.SSTA_BF16))))
 cases.append(("read_status_null", call("ssta_read_device_status", None, None, None)))
 lib.ssta_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                            ctypes.c_void_p]

@@ -74,7 +74,7 @@ def test_host_validation_codes():
         "mask_misaligned_cnt": ALIGN, "attn_bf16_tile_not_128": UNSUP, "attn_no_workspace": WS,
         "attn_small_workspace": WS, "attn_null_q": INVALID, "attn_misaligned_o": ALIGN,
         "bwd_no_workspace": WS, "bwd_small_workspace": WS, "bwd_ws_misaligned": ALIGN, "bwd_null_do": INVALID,
-        "bwd_misaligned_dk": ALIGN, "bwd_bad_desc": INVALID,
+        "bwd_misaligned_dk": ALIGN, "bwd_bad_desc": INVALID, "bwd_bf16_tile_not_128": UNSUP,
         "read_status_null": INVALID, "selftest_timeout_zero": INVALID, "selftest_timeout_huge": INVALID,
         "selftest_no_workspace": WS,
     }

@@ -21,10 +21,10 @@ the method states it.  Sources (page titles; sections / equations named):
       doubts the AND of Algorithm 1 and points to a union; the union is used).
 * "HunyuanVideo-1.5: An 8.3B-Parameter Video Diffusion Model Built for
   Consumer GPUs" (apoapsis blog), "Under the Hood: SSTA and Muon in Detail":
-  top-k is clamped to the number of key blocks; the importance-sampling
-  routine (pooled q and k normalised to unit length; similarity and key-key
-  terms mapped by (x + 1) / 2; the key-key diagonal excluded from the mean;
-  score = lambda * similarity - (1 - lambda) * redundancy, lambda = 0.9).
+  top-k is clamped to the number of key blocks; for the importance score it
+  fixes the constants of the report's Step 2 equation: lambda = 0.9 and
+  beta = 1 - lambda, cosines of the pooled vectors mapped by (x + 1) / 2, a
+  key tile not compared with itself in the redundancy.
 
 Modes (descriptor fields, defaults first): ``score_mode`` "similarity" (raw
 pooled dot product) or "importance" (Step 2's similarity-minus-redundancy
@@ -183,25 +183,35 @@ def _unit(x: np.ndarray) -> np.ndarray:
 
 
 def importance_scores(d, qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
-    """Step 2 with the redundancy term ("Selective Mask Generation": Score_i =
-    lambda Score_s - beta Score_r, Score_r the mean key-key similarity of a key
-    block to the other key blocks), in the blog's importance-sampling form:
-    pooled q and k normalised to unit length, similarity (q.k + 1) / 2 and
-    key-key similarity (k.k' + 1) / 2, the redundancy of key tile j the mean of
-    the key-key similarities of j with every other key tile (diagonal
-    excluded; 0 when there is no other tile), score = lam * similarity -
-    (1 - lam) * redundancy.  float64 [B,H,NT,NT]."""
+    """Step 2 with the redundancy term ("Selective Mask Generation"): the block
+    score Score_i = lam * Score_s - beta * Score_r, per (batch, head), with
+    beta = 1 - lam and lam = 0.9 by default (the weights the blog fixes).
+
+    * Score_s[i, j]: similarity of query tile i and key tile j, the cosine of
+      their pooled vectors mapped from [-1, 1] to [0, 1] by (x + 1) / 2;
+    * Score_r[j]: redundancy of key tile j, the average of the same mapped
+      cosine between key tile j and each OTHER key tile (a tile is not
+      compared with itself; with a single key tile there is no other tile and
+      Score_r = 0).
+
+    A pooled vector of length zero has cosine 0 with everything (its unit
+    vector is taken as zero).  float64 [B,H,NT,NT]."""
     lam = float(getattr(d, "lam", 0.9))
-    qn, kn = _unit(qbar), _unit(kbar)
-    sim = (np.einsum("bhid,bhjd->bhij", qn, kn) + 1.0) / 2.0
-    kk = (np.einsum("bhad,bhjd->bhaj", kn, kn) + 1.0) / 2.0      # [.., a, j]: key a vs key j
-    NT = kk.shape[-1]
-    off = ~np.eye(NT, dtype=bool)
-    if NT > 1:
-        red = (kk * off).sum(axis=-2) / (NT - 1)                # mean over a != j
-    else:
-        red = np.zeros(kk.shape[:-2] + (NT,))
-    return lam * sim - (1.0 - lam) * red[..., None, :]
+    beta = 1.0 - lam
+    B, H, NTq, NTk = qbar.shape[0], qbar.shape[1], qbar.shape[2], kbar.shape[2]
+    out = np.empty((B, H, NTq, NTk))
+    for b in range(B):
+        for h in range(H):
+            qn, kn = _unit(qbar[b, h]), _unit(kbar[b, h])
+            score_s = (qn @ kn.T + 1.0) / 2.0                     # [query tile, key tile]
+            score_r = np.zeros(NTk)
+            for j in range(NTk):
+                if NTk == 1:
+                    break
+                to_all = (kn @ kn[j] + 1.0) / 2.0                # key tile j against every key tile
+                score_r[j] = np.delete(to_all, j).mean()          # ... the other ones only
+            out[b, h] = lam * score_s - beta * score_r[None, :]
+    return out
 
 
 def block_scores(d, qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:

@@ -21,6 +21,10 @@
   single tile and all-zero vectors; top-k on them by brute force;
 * truncated window: brute force over each axis and the pages' |c' - c| <= w/2
   rule; AND combination: set intersection, and its two degenerate cases;
+* compact lists: a hand-built mask with out-of-order, full and empty rows
+  against hand-written ascending, -1-padded lists;
+* kept-block FLOP count: closed forms N^2 / v^2 for one partially valid tile
+  and (rows + text rows)^2 with a partial text tile, padded and valid-only;
 * backward (dQ, dK, dV): torch autograd through the float64 masked SDPA on the
   raster tokens (random kept sets with and without text, the dense case), the
   invariants sum_keys dV = sum_rows dO and sum_keys dK = 0, empty kept sets.
@@ -381,6 +385,51 @@ def test_flop_count_dense_case():
     kept = np.ones((1, w.H, g.NQ, g.NQ), dtype=bool)
     L = w.T * w.Y * w.X
     assert oracle.attention_flops(w, kept) == 4.0 * w.D * w.H * L * L
+
+
+def test_flop_count_partial_tiles_closed_form():
+    # one video tile of N = 4*8*8 = 256 slots holding a 3x5x2 grid (v = 30 valid tokens):
+    # padded it counts N x N (query row, key) pairs, valid-only v x v
+    d = _desc(T=3, Y=5, X=2, tT=4, tY=8, tX=8, topk=1, D=16, H=1)
+    kept = np.ones((1, 1, 1, 1), dtype=bool)
+    assert oracle.attention_flops(d, kept) == 4.0 * 16 * 256 * 256
+    assert oracle.attention_flops(d, kept, padded=False) == 4.0 * 16 * 30 * 30
+    # a 2x2x1 grid in 2x2x2 tiles (4 of 8 slots valid) plus 5 text tokens (one partial text
+    # tile): every pair kept; padded rows (8 video, 5 text) give (8 + 5)^2 pairs, valid rows
+    # (4 video, 5 text) give (4 + 5)^2
+    d = _desc(T=2, Y=2, X=1, tT=2, tY=2, tX=2, topk=1, L_text=5, D=8, H=3)
+    g = oracle.geometry(d)
+    assert (g.NT, g.n_text, g.NQ) == (1, 1, 2)
+    kept = np.ones((1, 3, 2, 2), dtype=bool)
+    assert oracle.attention_flops(d, kept) == 4.0 * 8 * 3 * 13 ** 2
+    assert oracle.attention_flops(d, kept, padded=False) == 4.0 * 8 * 3 * 9 ** 2
+    # drop the video query tile's text key tile in head 1: that head loses 8 x 5 padded and
+    # 4 x 5 valid pairs
+    kept[0, 1, 0, 1] = False
+    assert oracle.attention_flops(d, kept) == 4.0 * 8 * (3 * 169 - 40)
+    assert oracle.attention_flops(d, kept, padded=False) == 4.0 * 8 * (3 * 81 - 20)
+
+
+def test_kept_lists_of_a_hand_built_mask():
+    kept = np.zeros((1, 2, 3, 6), dtype=bool)
+    kept[0, 0, 0, [4, 1, 3]] = True            # set out of order: the list is ascending
+    kept[0, 0, 2, :] = True                    # every tile
+    kept[0, 1, 1, [5]] = True                  # row 0 of head 1 and row 1 of head 0 keep nothing
+    idx, cnt = oracle.kept_lists(kept)
+    assert idx.dtype == np.int32 and cnt.dtype == np.int32
+    want_idx = np.full((1, 2, 3, 6), -1, dtype=np.int32)            # width = the largest count, 6
+    want_idx[0, 0, 0, :3] = [1, 3, 4]
+    want_idx[0, 0, 2, :] = [0, 1, 2, 3, 4, 5]
+    want_idx[0, 1, 1, :1] = [5]
+    np.testing.assert_array_equal(idx, want_idx)
+    np.testing.assert_array_equal(cnt, [[[3, 0, 6], [0, 1, 0]]])
+    # width follows the largest count; an all-empty mask gives width 0
+    idx, cnt = oracle.kept_lists(kept[:, :, :2])
+    assert idx.shape == (1, 2, 2, 3)
+    np.testing.assert_array_equal(idx[0, 0, 0], [1, 3, 4])
+    np.testing.assert_array_equal(idx[0, 1, 1], [5, -1, -1])
+    idx, cnt = oracle.kept_lists(np.zeros((1, 1, 2, 4), dtype=bool))
+    assert idx.shape == (1, 1, 2, 0) and cnt.tolist() == [[[0, 0]]]
 
 
 # ---------------------------------------------------------------------------

@@ -157,6 +157,31 @@ def kept_flops(w, plan, kv_idx, kv_cnt):
     return padded, valid
 
 
+def issued_flops(w, plan, kv_idx):
+    """FLOPs the tensor-core attention kernel issues for one problem: every query tile
+    is computed on all N of its rows (128-row halves), and a kept key tile on each of
+    its 128-key chunks that holds at least one valid key (pad-only chunks are skipped).
+    4*D*N*128 per (query tile, kept chunk)."""
+    import numpy as np
+    N = plan.tile_tokens
+    nT, nY, nX = -(-w.T // w.tT), -(-w.Y // w.tY), -(-w.X // w.tX)
+    o = np.arange(N)
+    dt, dy, dx = o // (w.tX * w.tY), (o // w.tX) % w.tY, o % w.tX
+    vt = np.minimum(w.tT, w.T - np.arange(nT) * w.tT)
+    vy = np.minimum(w.tY, w.Y - np.arange(nY) * w.tY)
+    vx = np.minimum(w.tX, w.X - np.arange(nX) * w.tX)
+    valid = ((dt[None, None, None, :] < vt[:, None, None, None]) & (dy[None, None, None, :] < vy[None, :, None, None])
+             & (dx[None, None, None, :] < vx[None, None, :, None])).reshape(-1, N // 128, 128)
+    chunks = valid.any(-1).sum(-1).astype(np.float64)                       # [NT]
+    if plan.num_text_tiles:
+        rem = w.L_text - np.arange(plan.num_text_tiles) * N
+        chunks = np.concatenate([chunks, np.ceil(np.minimum(rem, N) / 128.0)])
+    idx = kv_idx.cpu().numpy()
+    ok = idx >= 0
+    per_row = np.where(ok, chunks[np.where(ok, idx, 0)], 0.0).sum(-1)       # kept chunks per query tile
+    return 4.0 * w.D * N * 128.0 * float(per_row.sum())
+
+
 def pci_bus_id(dev):
     import torch
     p = torch.cuda.get_device_properties(dev)
@@ -366,6 +391,8 @@ def run_gpu(args):
         if st != (0, 0):
             raise RuntimeError(f"device status {st}")
     flops = [kept_flops(w, plan, p["kv_idx"], p["kv_cnt"]) for p in probs]
+    issued = [issued_flops(w, plan, p["kv_idx"]) if (w.dtype == "bf16" and plan.tile_tokens % 128 == 0) else None
+              for p in probs]
 
     # ---- timed region (device-resident inputs)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
@@ -383,6 +410,31 @@ def run_gpu(args):
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     stage = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])   # [K, 4]
+    # ---- L2 flushed vs warm samples, outside the timed region: the mask build 20 times with
+    # a 256 MB write (twice the L2) before each sample, the attention 3 times flushed and 3
+    # times right after a run on the same inputs (warm); medians.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    p0 = probs[0]
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, pre=None):
+        if pre is not None:
+            pre()
+        e_a.record(stream)
+        fn()
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        return e_a.elapsed_time(e_b)
+
+    mask_call = lambda: S.ssta_build_block_mask(d, p0["qp"], p0["kp"], p0["kv_idx"], p0["kv_cnt"], workspace=p0["ws"])
+    attn_call = lambda: S.ssta_attention_fwd(d, p0["qp"], p0["kp"], p0["vp"], p0["kv_idx"], p0["kv_cnt"], p0["op"],
+                                             p0["lse"], workspace=p0["ws_a"])
+    mask_flushed = statistics.median(timed(mask_call, flush.zero_) for _ in range(20))
+    mask_warm = statistics.median(timed(mask_call, mask_call) for _ in range(20))
+    attn_flushed = statistics.median(timed(attn_call, flush.zero_) for _ in range(3))
+    attn_warm = statistics.median(timed(attn_call, attn_call) for _ in range(3))
+    del flush
+
     my_flops = sum(flops[i % len(probs)][0] for i in range(args.steps))
     my_vflops = sum(flops[i % len(probs)][1] for i in range(args.steps))
     attn_flops = my_flops
@@ -449,12 +501,15 @@ def run_gpu(args):
 
     if rank == 0:
         peaks, src = load_peaks()
-        attn_ms = float(stage[:, 2].mean())
-        mask_ms = float(stage[:, 1].mean())
-        reorder_ms = float(stage[:, 0].mean())
-        unorder_ms = float(stage[:, 3].mean())
+        attn_ms = float(np.median(stage[:, 2]))
+        mask_ms = float(np.median(stage[:, 1]))
+        reorder_ms = float(np.median(stage[:, 0]))
+        unorder_ms = float(np.median(stage[:, 3]))
+        attn_ms_mean = float(stage[:, 2].mean())
         per_call_flops = attn_flops / args.steps
-        achieved = per_call_flops / (attn_ms / 1000.0) / 1e12
+        achieved = per_call_flops / (attn_ms_mean / 1000.0) / 1e12
+        per_call_issued = (sum(issued[i % len(probs)] for i in range(args.steps)) / args.steps
+                           if issued[0] is not None else None)
         peak_sus = float(peaks["bf16_tflops_sustained"])
         peak_burst = float(peaks["bf16_tflops"])
         hbm = float(peaks["hbm_gbs"])
@@ -481,15 +536,31 @@ def run_gpu(args):
                        "parallelism": f"dp{world} (one independent problem per rank)",
                        "l2": "no flush: every input tensor (0.9-1.0 GB) is larger than the 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": "ssta_attention_tc_kernel", "achieved": achieved,
-                         "peak": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak_sus,
-                         "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
-                         "frac_of_burst_peak": achieved / peak_burst,
+                         "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved / peak_burst,
+                         "peak_source": (f"{src} bf16_tflops (burst: the kernel runs at the SM clock of "
+                                         f"'clocks', not at the power-capped clock of the sustained figure)"),
+                         "work": "kept-block FLOPs per launch (4*D*rows*rows per kept tile pair, tiles as laid "
+                                 "out) / mean CUDA-event duration of the launch",
+                         "frac_of_sustained_peak": achieved / peak_sus,
+                         "issued_tflop_per_call": None if per_call_issued is None else per_call_issued / 1e12,
+                         "issued_achieved": (None if per_call_issued is None
+                                             else per_call_issued / (attn_ms_mean / 1000.0) / 1e12),
+                         "issued_frac": (None if per_call_issued is None
+                                         else per_call_issued / (attn_ms_mean / 1000.0) / 1e12 / peak_burst),
                          "traffic": load_traffic("ssta_attn_tc.cu", w.name)},
             "stages_ms": {"tile_reorder_qkv": reorder_ms, "build_block_mask": mask_ms, "attention_fwd": attn_ms,
-                          "tile_unorder_o": unorder_ms},
+                          "tile_unorder_o": unorder_ms, "statistic": f"median of {args.steps} steps",
+                          "attention_fwd_mean": attn_ms_mean},
+            "l2_samples_ms": {"build_block_mask_flushed": mask_flushed, "build_block_mask_warm": mask_warm,
+                              "attention_fwd_flushed": attn_flushed, "attention_fwd_warm": attn_warm,
+                              "how": "outside the timed region, seed " + str(seeds[0]) + ": 256 MB written "
+                                     "before each flushed sample; warm = right after a run on the same inputs; "
+                                     "medians of 20 (mask) and 3 (attention)"},
             "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": hbm, "unit": "GB/s",
                               "frac": mask_gbs / hbm, "algorithmic_bytes": mask_bytes,
-                              "peak_source": f"{src} hbm_gbs"},
+                              "peak_source": f"{src} hbm_gbs",
+                              "flushed_achieved": mask_bytes / (mask_flushed / 1000.0) / 1e9,
+                              "flushed_frac": mask_bytes / (mask_flushed / 1000.0) / 1e9 / hbm},
             "reorder_gbs": (reorder_bytes / (reorder_ms / 1000.0) / 1e9),
             "kept_tflop_per_call": per_call_flops / 1e12,
             "valid_tflop_per_call": (my_vflops / args.steps) / 1e12,

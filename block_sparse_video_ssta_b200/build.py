@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import argparse
 import concurrent.futures as cf
+import hashlib
 import os
 import shutil
 import subprocess
@@ -20,6 +21,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(HERE, "libssta.so")
+STAMP = OUT + ".sha256"   # hash of the sources the library was built from
 BUILD_DIR = os.path.join(ROOT, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -37,13 +39,26 @@ def sources():
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _needs_rebuild() -> bool:
-    if not os.path.exists(OUT):
-        return True
-    t = os.path.getmtime(OUT)
-    deps = sources() + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
+def _source_hash(extra_flags=()) -> str:
+    """sha256 over every source and header the library is built from, and the flags."""
+    h = hashlib.sha256()
+    deps = sources() + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh")))
     deps.append(os.path.join(INCLUDE, "ssta.h"))
-    return any(os.path.getmtime(p) > t for p in deps)
+    for p in deps:
+        h.update(os.path.relpath(p, ROOT).encode() + b"\0")
+        with open(p, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(ARCH + FLAGS[:-4] + list(extra_flags)).encode())
+    return h.hexdigest()
+
+
+def _needs_rebuild() -> bool:
+    """Rebuild unless the library exists and its stamp holds the current sources' hash
+    (file times are not trusted: a copied tree can carry a library newer than its sources)."""
+    if not (os.path.exists(OUT) and os.path.exists(STAMP)):
+        return True
+    with open(STAMP) as f:
+        return f.read().strip() != _source_hash()
 
 
 def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) -> str:
@@ -77,6 +92,8 @@ def build(verbose: bool = False, force: bool = False, ptxas_info: bool = False) 
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("link failed")
     os.replace(tmp, OUT)
+    with open(STAMP, "w") as f:
+        f.write(_source_hash() + "\n")
     return OUT
 
 

@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "ssta_internal.h"
 
 namespace ssta {
@@ -14,7 +16,14 @@ constexpr int kMaxTiles = 2048;        // NT; one warp holds a score row in regi
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-ssta_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH; }
+// NVTX range over one library call (host side: validation and kernel enqueue), so a
+// timeline tool shows each call by name; without a tool attached it costs a few ns.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 }  // namespace
 
@@ -102,6 +111,7 @@ ssta_status ssta_plan(const ssta_desc* desc, ssta_plan_info* info) {
 
 ssta_status ssta_tile_reorder(const ssta_desc* desc, const void* x_raster, const void* x_text, void* x_packed,
                               void* stream) {
+  NvtxRange nvtx("ssta_tile_reorder");
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
@@ -116,6 +126,7 @@ ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, cons
                                const void* v_packed, const void* o_packed, const float* lse, const void* do_packed,
                                const int32_t* kv_idx, const int32_t* kv_cnt, void* dq_packed, void* dk_packed,
                                void* dv_packed, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx("ssta_attention_bwd");
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
@@ -138,6 +149,7 @@ ssta_status ssta_attention_bwd(const ssta_desc* desc, const void* q_packed, cons
 
 ssta_status ssta_tile_unorder(const ssta_desc* desc, const void* x_packed, void* x_raster, void* x_text,
                               void* stream) {
+  NvtxRange nvtx("ssta_tile_unorder");
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
@@ -151,6 +163,7 @@ ssta_status ssta_tile_unorder(const ssta_desc* desc, const void* x_packed, void*
 ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, const void* k_packed,
                                   int32_t* kv_idx, int32_t* kv_cnt, float* tile_scores, void* workspace,
                                   size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx("ssta_build_block_mask");
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;
@@ -184,6 +197,7 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
 ssta_status ssta_attention_fwd(const ssta_desc* desc, const void* q_packed, const void* k_packed,
                                const void* v_packed, const int32_t* kv_idx, const int32_t* kv_cnt, void* o_packed,
                                float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx("ssta_attention_fwd");
   Geom g;
   ssta_status st = make_geom(desc, &g);
   if (st != SSTA_OK) return st;

@@ -108,6 +108,9 @@ cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* 
 // Device-side helpers shared by kernels.
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Status of a host-side CUDA runtime call (a launch, a memset): SSTA_ERR_LAUNCH on any error.
+inline ssta_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH; }
+
 // Number of valid tokens along one axis of tile coordinate c (tile extent t, valid extent n).
 __host__ __device__ inline int axis_valid(int c, int t, int n) {
   int v = n - c * t;

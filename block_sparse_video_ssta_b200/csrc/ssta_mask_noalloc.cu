@@ -13,8 +13,10 @@
 //  * the array (SSTA_STATIC_SCRATCH_BYTES) exists on every GPU that loads this
 //    library and stays resident until the process exits;
 //  * every call on a device uses the same array, which keeps the contents of
-//    the last call: the status word is cleared on every call, and every other
-//    region is fully rewritten before it is read;
+//    the last call: every region is fully rewritten before it is read;
+//  * the mask kernels report no device-side errors (their inputs are checked
+//    on the host), and the array's address is not exported, so this call keeps
+//    no device status word: its first bytes stay unused;
 //  * calls whose kernels overlap on the GPU (different streams, or different
 //    host threads, on the same device) race on the array: serialise them;
 //  * in host code the array's name is only a host-side stand-in, so its device
@@ -77,7 +79,7 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   if (st != SSTA_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(base_v);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (empty) return cudaMemsetAsync(base, 0, sizeof(int32_t), s) == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;
+  if (empty) return SSTA_OK;
   float* qbar = reinterpret_cast<float*>(base + ws.qbar);
   float* kbar = reinterpret_cast<float*>(base + ws.kbar);
   float* scores = tile_scores != nullptr ? tile_scores : reinterpret_cast<float*>(base + ws.scores);
@@ -85,10 +87,10 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   const ImportanceBufs ib = imp ? ImportanceBufs{reinterpret_cast<float*>(base + ws.inv_nq), reinterpret_cast<float*>(base + ws.inv_nk),
                                                  reinterpret_cast<float*>(base + ws.ksum)}
                                 : ImportanceBufs{nullptr, nullptr, nullptr};
-  // the pool kernel also clears the status word
-  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(base + ws.status), ib, s);
+  // no status word (nullptr): nothing could read it back
+  cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, nullptr, ib, s);
   if (e == cudaSuccess && imp) e = launch_tile_keysum(g, kbar, ib, s);
   if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
-  return e == cudaSuccess ? SSTA_OK : SSTA_ERR_LAUNCH;
+  return from_cuda(e);
 }

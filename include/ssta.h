@@ -227,9 +227,13 @@ ssta_status ssta_tile_unorder(const ssta_desc* desc, const void* x_packed, void*
  * tensors, or a service that reserved all device memory for its own pool).  The
  * paper has no counterpart to this call; it exists for those callers only.
  *   Scratch: a device array of SSTA_STATIC_SCRATCH_BYTES built into the library,
- *   one per GPU that loads it, resident until the process exits.  Problems whose
- *   scratch would exceed it (status word, pooled q and k, the score matrix
- *   unless tile_scores is given, selection bits) return SSTA_ERR_WORKSPACE.
+ *   one per GPU that loads it, resident until the process exits.  It holds the
+ *   workspace layout of ssta_build_block_mask: a 256-byte header, the pooled q and
+ *   k means, in importance mode the inverse norms and the key sums, and the score
+ *   matrix unless tile_scores is given.  Problems whose layout exceeds the array
+ *   return SSTA_ERR_WORKSPACE.  The mask kernels report no device-side errors and
+ *   the array's address is not exported, so this call keeps no device status word
+ *   (there is nothing for ssta_read_device_status to read).
  *   The call allocates nothing.  All calls on a device share the array, so calls
  *   whose kernels overlap on the GPU race: serialise them.  The first call on a
  *   device looks up the array's device address (with that device current); make

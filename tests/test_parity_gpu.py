@@ -13,7 +13,7 @@ import block_sparse_video_ssta_b200 as S
 import oracle
 import ssta_inputs as si
 from ssta_inputs import with_overrides
-from ssta_parity import full_check, gpu_kept, run_gpu, to_np
+from ssta_parity import full_check, gpu_kept, mask_check, run_gpu, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -121,6 +121,18 @@ def test_full_size_sampled(cuda_ok, name):
     w = si.get_workload(name)
     st = full_check(w, seed=0, q_tiles=_sampled(w), heads=[0, w.H // 2, w.H - 1])
     _report(name, st)
+    g = oracle.geometry(w)
+    assert st["rows_mask_mismatch"] <= max(2, g.NT // 100)
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_p720_10s_masks_other_seeds(cuda_ok, seed):
+    """The benchmark cycles the 720p 10 s workload over seeds 0-2: packing, scores and
+    kept lists of seeds 1 and 2 against the oracle on every mask row of three heads
+    (seed 0 is covered with attention by test_full_size_sampled)."""
+    w = si.get_workload("p720_10s_bf16")
+    st = mask_check(w, seed, heads=[1, w.H // 2 + 1, w.H - 2])
+    _report(f"p720_10s seed {seed} masks", st)
     g = oracle.geometry(w)
     assert st["rows_mask_mismatch"] <= max(2, g.NT // 100)
 

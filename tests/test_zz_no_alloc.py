@@ -29,7 +29,8 @@ def _stream():
 @pytest.mark.parametrize("name,with_scores,mode", [("tiny_f32", True, "similarity"), ("small_bf16", False, "similarity"),
                                                    ("small_bf16", True, "similarity"),
                                                    ("p720_5s_bf16", False, "similarity"),
-                                                   ("small_bf16", False, "importance")])
+                                                   ("small_bf16", False, "importance"),
+                                                   ("small_bf16", True, "importance")])
 def test_noalloc_matches_workspace_entry_point(cuda_ok, name, with_scores, mode):
     w = si.with_overrides(si.get_workload(name), score_mode=mode)
     x = si.make_inputs(w, 2, device="cuda")

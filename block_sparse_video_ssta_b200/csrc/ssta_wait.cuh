@@ -46,9 +46,10 @@ struct Ctl {
   uint64_t timeout_ns;        // limit of one wait
 };
 
-// Bounded wait by one thread.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Polling loop of a bounded wait, entered only when the first try_wait gave up.  Kept
+// out of line: a call costs a few hundred clocks (the caller's live registers go to the
+// stack), which is why the first try sits inline in wait_bounded.
+__device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
   const uint64_t t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -59,6 +60,12 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const C
       return false;
     }
   }
+}
+// Bounded wait by one thread: one inline try_wait (which itself blocks in hardware for a
+// while and returns as soon as the phase completes), then the polling loop.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bounded_slow(bar, parity, c);
 }
 // Bounded wait by a whole warp; the outcome is made warp-uniform.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const Ctl& c) {

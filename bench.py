@@ -46,8 +46,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def load_traffic(kernel_file, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
+def load_traffic(kernel_file, w):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel
+    source and on this workload (name and head count)."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -57,7 +58,7 @@ def load_traffic(kernel_file, workload):
     src = os.path.join(ROOT, "block_sparse_video_ssta_b200", "csrc", kernel_file)
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     e = d.get(kernel_file, {})
-    if e.get("source_sha256_16") == h and e.get("workload") == workload:
+    if e.get("source_sha256_16") == h and e.get("workload") == w.name and e.get("heads", 16) == w.H:
         return e.get("dram_bytes_per_launch")
     return None
 
@@ -295,7 +296,7 @@ def workload_of(args):
     import ssta_inputs as si
     w = si.get_workload(args.workload)
     ov = {k: v for k, v in (("score_mode", args.score_mode), ("combine", args.combine),
-                            ("window_mode", args.window_mode)) if v is not None}
+                            ("window_mode", args.window_mode), ("H", args.heads)) if v is not None}
     return si.with_overrides(w, **ov) if ov else w
 
 
@@ -547,7 +548,7 @@ def run_gpu(args):
                                              else per_call_issued / (attn_ms_mean / 1000.0) / 1e12),
                          "issued_frac": (None if per_call_issued is None
                                          else per_call_issued / (attn_ms_mean / 1000.0) / 1e12 / peak_burst),
-                         "traffic": load_traffic("ssta_attn_tc.cu", w.name)},
+                         "traffic": load_traffic("ssta_attn_tc.cu", w)},
             "stages_ms": {"tile_reorder_qkv": reorder_ms, "build_block_mask": mask_ms, "attention_fwd": attn_ms,
                           "tile_unorder_o": unorder_ms, "statistic": f"median of {args.steps} steps",
                           "attention_fwd_mean": attn_ms_mean},
@@ -643,6 +644,8 @@ def main():
                     help="block score ranked by top-k (default: the workload's, similarity)")
     ap.add_argument("--combine", default=None, choices=["union", "and"])
     ap.add_argument("--window-mode", default=None, choices=["shift", "truncate"])
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with this many heads (small profiling cases; not a headline run)")
     ap.add_argument("--backward", action="store_true",
                     help="time ssta_attention_bwd instead of the forward (prints its own line)")
     args = ap.parse_args()

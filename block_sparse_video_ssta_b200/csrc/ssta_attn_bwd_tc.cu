@@ -55,7 +55,7 @@ enum : int {
 __global__ void __launch_bounds__(kDqThreads, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Geom g,
-                 const ChunkTables tb, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
+                 const __grid_constant__ ChunkTables tb, const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
                  const float* __restrict__ lse, const float* __restrict__ Dv, __nv_bfloat16* __restrict__ dq,
                  int32_t* __restrict__ status, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
@@ -225,7 +225,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int r = grp * 32 + lane;   // row within the block
     const int64_t row = (int64_t)qrow0 + r;
     const int qoff = (int)(row - (int64_t)qt * g.N);
-    const bool row_ok = row < g.Lq && key_valid(g, qt, qoff);
+    const bool row_ok = row < g.Lq && key_valid(g, tb, qt, qoff);
     const float L2 = row_ok ? __ldg(lse + bh * g.Lq + row) * 1.4426950408889634f : 0.f;
     const bool live = row_ok && L2 > -INFINITY;
     const float Dr = live ? __ldg(Dv + bh * g.Lq + row) : 0.f;
@@ -240,8 +240,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_arrive(bar(BAR_SFREE));   // S and dP of this chunk are in registers
       uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;   // valid keys of columns [0,32), [32,64) of this half
       if (!full) {
-        vm0 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + lane));
-        vm1 = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + 64 * half + 32 + lane));
+        vm0 = chunk_vmask(g, tb, t, ch, 2 * half);
+        vm1 = chunk_vmask(g, tb, t, ch, 2 * half + 1);
       }
       uint32_t pk[32];
 #pragma unroll
@@ -397,7 +397,7 @@ __device__ __forceinline__ int for_each_qchunk(const Geom& g, const ChunkTables&
 __global__ void __launch_bounds__(kKvThreads, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Geom g,
-                   const ChunkTables tb, const int32_t* __restrict__ tidx, const int32_t* __restrict__ tcnt,
+                   const __grid_constant__ ChunkTables tb, const int32_t* __restrict__ tidx, const int32_t* __restrict__ tcnt,
                    const float* __restrict__ lse, const float* __restrict__ Dv, __nv_bfloat16* __restrict__ dk,
                    __nv_bfloat16* __restrict__ dv, int32_t* __restrict__ status, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
@@ -504,7 +504,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int i = 0; i < 4; ++i) {
         const int c = lane + 32 * i;
         const int64_t row = (int64_t)qrow + c;
-        const bool ok = row < g.Lq && key_valid(g, t, ch * kChunk + c);
+        const bool ok = row < g.Lq && key_valid(g, tb, t, ch * kChunk + c);
         const float L = ok ? __ldg(lse + bh * g.Lq + row) : -INFINITY;
         l2[c] = L > -INFINITY ? L * 1.4426950408889634f : INFINITY;   // +inf: the row contributes nothing
         dd[c] = L > -INFINITY ? __ldg(Dv + bh * g.Lq + row) : 0.f;
@@ -569,7 +569,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int grp = warp & 3, half = warp >> 2;
     const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
     const int64_t row = (int64_t)krow0 + grp * 32 + lane;
-    const bool key_ok = row < g.Lq && key_valid(g, kt, (int)(row - (int64_t)kt * g.N));
+    const bool key_ok = row < g.Lq && key_valid(g, tb, kt, (int)(row - (int64_t)kt * g.N));
     const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
       if (!wait_warp(bar(KB_SFULL), (uint32_t)(step & 1), ctl)) return false;
       // the producer's per-query values of this stage: acquire them from its own barrier

@@ -70,7 +70,7 @@ constexpr uint32_t kIdescPV = kIdescKMN;
 // ------------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(kThreads, 1)
 ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                         const __grid_constant__ CUtensorMap tmV, const Geom g, const ChunkTables tb,
+                         const __grid_constant__ CUtensorMap tmV, const Geom g, const __grid_constant__ ChunkTables tb,
                          const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt,
                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t* __restrict__ status,
                          float scale_log2) {
@@ -274,7 +274,7 @@ ssta_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         // pad keys of this chunk (same columns for every row) never enter the softmax
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint32_t vm = __ballot_sync(0xffffffffu, key_valid(g, t, ch * kChunk + q * 32 + lane));
+          const uint32_t vm = chunk_vmask(g, tb, t, ch, q);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (!((vm >> i) & 1u)) sv[q * 32 + i] = -INFINITY;

@@ -29,12 +29,22 @@ constexpr uint32_t kTileBytes = 2 * kBox;           // 128 rows x 128 channels
 constexpr uint32_t kIdescKK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescKMN = kIdescKK | (1u << 16);
 
-// Which 128-key chunks of a tile hold at least one valid key / only valid keys,
-// for the 8 classes of video tiles (bit 2: last along T with padding, bit 1:
-// last along Y, bit 0: last along X).  Bit c of a word = chunk c.
+// Tile geometry as lookup tables, passed to the kernels as a __grid_constant__
+// parameter (read through the constant cache; every index used is warp-uniform).
+// A video tile belongs to one of 8 classes (bit 2: last along T with padding,
+// bit 1: last along Y, bit 0: last along X); text tiles are handled arithmetically.
+//   any / full[cls]   bit c: 128-key chunk c holds at least one / only valid keys
+//   vmask[cls][c][w]  bit b: key 128c + 32w + b of the tile is valid
+//   cls[t]            class of video tile t
+// Divisions by the grid extents (which go through the XU pipe next to the
+// softmax exponentials) are thus taken once, on the host.
+constexpr int kMaxTileChunks = 32;     // N <= 4096 tokens per tile
+constexpr int kMaxVideoTiles = 2048;   // NT limit of the library
 struct ChunkTables {
   uint32_t any[8];
   uint32_t full[8];
+  uint32_t vmask[8][kMaxTileChunks][4];
+  uint8_t cls[kMaxVideoTiles];
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -174,22 +184,24 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr) {
 // ------------------------------------------------------------- chunk sequence
 __device__ __forceinline__ void chunk_bits(const Geom& g, const ChunkTables& tb, int t, uint32_t& any,
                                            uint32_t& full) {
-  const int nch = g.N / kChunk;
   if (t < g.NT) {
-    const int cX = t % g.nX, cY = (t / g.nX) % g.nY, cT = t / (g.nX * g.nY);
-    const int cls = ((cT == g.nT - 1 && g.T % g.tT) ? 4 : 0) | ((cY == g.nY - 1 && g.Y % g.tY) ? 2 : 0) |
-                    ((cX == g.nX - 1 && g.X % g.tX) ? 1 : 0);
+    const int cls = tb.cls[t];
     any = tb.any[cls];
     full = tb.full[cls];
   } else {
+    const int nch = g.N / kChunk;
     const int rem = g.L_text - (t - g.NT) * g.N;   // valid keys in this text tile
-    any = 0;
-    full = 0;
-    for (int c = 0; c < nch; ++c) {
-      if (c * kChunk < rem) any |= 1u << c;
-      if ((c + 1) * kChunk <= rem) full |= 1u << c;
-    }
+    const int nany = min(nch, (rem + kChunk - 1) / kChunk), nfull = min(nch, rem / kChunk);
+    any = nany >= 32 ? 0xffffffffu : ((1u << nany) - 1u);
+    full = nfull >= 32 ? 0xffffffffu : ((1u << nfull) - 1u);
   }
+}
+
+// Valid keys 32w .. 32w + 31 of chunk ch of tile t, one bit each.
+__device__ __forceinline__ uint32_t chunk_vmask(const Geom& g, const ChunkTables& tb, int t, int ch, int w) {
+  if (t < g.NT) return tb.vmask[tb.cls[t]][ch][w];
+  const int rem = g.L_text - (t - g.NT) * g.N - ch * kChunk - 32 * w;   // valid keys from key 32w on
+  return rem >= 32 ? 0xffffffffu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
 }
 
 // Calls f(j, t, ch, full) for every chunk with a valid key, in list order; stops
@@ -213,13 +225,9 @@ __device__ __forceinline__ int for_each_chunk(const Geom& g, const ChunkTables& 
   return j;
 }
 
-__device__ __forceinline__ bool key_valid(const Geom& g, int t, int o) {
-  if (t < g.NT) {
-    const int cX = t % g.nX, cY = (t / g.nX) % g.nY, cT = t / (g.nX * g.nY);
-    const int dx = o % g.tX, dy = (o / g.tX) % g.tY, dt = o / (g.tX * g.tY);
-    return dt < axis_valid(cT, g.tT, g.T) && dy < axis_valid(cY, g.tY, g.Y) && dx < axis_valid(cX, g.tX, g.X);
-  }
-  return (t - g.NT) * g.N + o < g.L_text;
+// Whether token o (0 <= o < N) of tile t is a real (non-pad) token.
+__device__ __forceinline__ bool key_valid(const Geom& g, const ChunkTables& tb, int t, int o) {
+  return (chunk_vmask(g, tb, t, o >> 7, (o >> 5) & 3) >> (o & 31)) & 1u;
 }
 
 
@@ -272,6 +280,7 @@ bool make_map(CUtensorMap* map, const void* ptr, const Geom& g) {
   return r == CUDA_SUCCESS;
 }
 
+// Host side.  Requires N % 128 == 0, N <= 4096 and NT <= 2048 (checked by the API).
 ChunkTables make_chunk_tables(const Geom& g) {
   ChunkTables tb{};
   const int nch = g.N / kChunk;
@@ -279,15 +288,22 @@ ChunkTables make_chunk_tables(const Geom& g) {
     const int vt = (cls & 4) ? g.T - (g.nT - 1) * g.tT : g.tT;
     const int vy = (cls & 2) ? g.Y - (g.nY - 1) * g.tY : g.tY;
     const int vx = (cls & 1) ? g.X - (g.nX - 1) * g.tX : g.tX;
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nch && c < kMaxTileChunks; ++c) {
       int valid = 0;
       for (int o = c * kChunk; o < (c + 1) * kChunk; ++o) {
         const int dx = o % g.tX, dy = (o / g.tX) % g.tY, dt = o / (g.tX * g.tY);
-        valid += (dt < vt && dy < vy && dx < vx) ? 1 : 0;
+        const bool ok = dt < vt && dy < vy && dx < vx;
+        valid += ok ? 1 : 0;
+        if (ok) tb.vmask[cls][c][(o - c * kChunk) >> 5] |= 1u << (o & 31);
       }
       if (valid > 0) tb.any[cls] |= 1u << c;
       if (valid == kChunk) tb.full[cls] |= 1u << c;
     }
+  }
+  for (int t = 0; t < g.NT && t < kMaxVideoTiles; ++t) {
+    const int cX = t % g.nX, cY = (t / g.nX) % g.nY, cT = t / (g.nX * g.nY);
+    tb.cls[t] = (uint8_t)(((cT == g.nT - 1 && g.T % g.tT) ? 4 : 0) | ((cY == g.nY - 1 && g.Y % g.tY) ? 2 : 0) |
+                          ((cX == g.nX - 1 && g.X % g.tX) ? 1 : 0));
   }
   return tb;
 }

@@ -1,5 +1,5 @@
-// tcgen05 / TMA building blocks shared by the tensor-core kernels of the
-// backward pass: PTX wrappers (mbarrier transaction counts, 3D TMA loads,
+// tcgen05 / TMA building blocks shared by the tensor-core kernels (the
+// attention forward and the two backward kernels): PTX wrappers (mbarrier transaction counts, 3D TMA loads,
 // tcgen05 MMA, commit, fences, TMEM loads and stores), shared-memory matrix
 // descriptors for 128-byte-swizzled bf16 tiles, the per-tile chunk tables and
 // chunk walk over a kept-tile list, and the host-side tensor-map encoding.

@@ -32,8 +32,12 @@
 
 #include <cuda_bf16.h>
 
+#include "ssta_f32x2.cuh"
+
 namespace ssta {
 namespace {
+
+using namespace f32x2;
 
 // Programmatic dependent launch: a kernel launched with launch_dependent() may start
 // while the previous kernel of the stream is still running; grid_dependency_wait()
@@ -204,21 +208,6 @@ tile_keysum_kernel(Geom g, const float* __restrict__ kbar_t, ImportanceBufs ib) 
 // past NT are zero-filled) into two buffers, so the next stage is in flight
 // while the current one is consumed.  Every score is accumulated over channels
 // 0..D-1 in order with FMA, two adjacent columns per fma.rn.f32x2 instruction.
-// Two-lane fp32 arithmetic (sm_100): one instruction for a pair of values, each
-// lane rounded exactly as the scalar instruction would.
-__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
 
 constexpr int kScoreBlock = 128;
 constexpr int kScoreStage = 16;   // channels per stage

@@ -229,6 +229,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const float L2 = row_ok ? __ldg(lse + bh * g.Lq + row) * 1.4426950408889634f : 0.f;
     const bool live = row_ok && L2 > -INFINITY;
     const float Dr = live ? __ldg(Dv + bh * g.Lq + row) : 0.f;
+    // per-row constants as f32x2 pairs: the scale, -LSE (log2 units; -inf for a row that takes
+    // no part, whose P is then exactly 0) and -D
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+    const float nl = live ? -L2 : -INFINITY;
+    const uint64_t nl2 = f2_pack(nl, nl), nd2 = f2_pack(-Dr, -Dr);
     uint8_t* ds_row = base_ptr + kOffDS + half * kBox + r * 128;   // this thread's 64 keys: one box row
     const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool full) -> bool {
       if (!wait_warp(bar(BAR_SFULL), (uint32_t)(j & 1), ctl)) return false;
@@ -238,23 +243,25 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_ld64(tP + lane_off + 64u * half, dpv);
       tc_fence_before();
       mbar_arrive(bar(BAR_SFREE));   // S and dP of this chunk are in registers
-      uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;   // valid keys of columns [0,32), [32,64) of this half
       if (!full) {
-        vm0 = chunk_vmask(g, tb, t, ch, 2 * half);
-        vm1 = chunk_vmask(g, tb, t, ch, 2 * half + 1);
+        // pad keys of this chunk (same columns for every row): S = -inf, so P = 0
+#pragma unroll
+        for (int w2 = 0; w2 < 2; ++w2) {
+          const uint32_t vm = chunk_vmask(g, tb, t, ch, 2 * half + w2);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (!((vm >> i) & 1u)) sv[32 * w2 + i] = -INFINITY;
+        }
       }
+      // P = 2^(s * scale - LSE), dS = P (dP - D), two key columns per f32x2 instruction
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        float ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 2 * i + e;
-          const bool kv = ((c < 32 ? vm0 >> c : vm1 >> (c - 32)) & 1u) != 0;
-          const float p = (live && kv) ? ex2(sv[c] * scale_log2 - L2) : 0.f;
-          ds[e] = p * (dpv[c] - Dr);
-        }
-        pk[i] = pack_bf16x2(ds[0], ds[1]);
+        float x0, x1, ds0, ds1;
+        f2_unpack(f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), c2, nl2), x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(dpv[2 * i], dpv[2 * i + 1]), nd2)), ds0, ds1);
+        pk[i] = pack_bf16x2(ds0, ds1);
       }
       // dQ(j-1) reads dS from shared memory: it must have finished before dS is overwritten
       if (j > 0 && !wait_warp(bar(BAR_DQDONE), (uint32_t)((j - 1) & 1), ctl)) return false;
@@ -506,8 +513,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int64_t row = (int64_t)qrow + c;
         const bool ok = row < g.Lq && key_valid(g, tb, t, ch * kChunk + c);
         const float L = ok ? __ldg(lse + bh * g.Lq + row) : -INFINITY;
-        l2[c] = L > -INFINITY ? L * 1.4426950408889634f : INFINITY;   // +inf: the row contributes nothing
-        dd[c] = L > -INFINITY ? __ldg(Dv + bh * g.Lq + row) : 0.f;
+        // negated, so the elementwise step adds them: -LSE in log2 units (-inf for a row without
+        // meaning, whose P is then exactly 0) and -D
+        l2[c] = L > -INFINITY ? -(L * 1.4426950408889634f) : -INFINITY;
+        dd[c] = L > -INFINITY ? -__ldg(Dv + bh * g.Lq + row) : 0.f;
       }
       mbar_arrive(bar(KB_QFULL + s));
       ++issued[s];
@@ -580,19 +589,23 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       float sv[64], dpv[64];
       tmem_ld64(tS + lane_off + 64u * half, sv);
       tmem_ld64(tP + lane_off + 64u * half, dpv);
+      // P = 2^(s * scale - LSE), dS = P (dP - D), two query columns per f32x2 instruction; the
+      // stage holds -LSE (log2 units, -inf for a row without meaning: P = 0) and -D
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2);
       uint32_t pkp[32], pks[32];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float4 L = reinterpret_cast<const float4*>(l2 + 64 * half)[i];
-        const float4 Dq = reinterpret_cast<const float4*>(dd + 64 * half)[i];
-        const float Ls[4] = {L.x, L.y, L.z, L.w}, Ds[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
-        float p[4], ds[4];
+        const float4 nl = reinterpret_cast<const float4*>(l2 + 64 * half)[i];
+        const float4 nd = reinterpret_cast<const float4*>(dd + 64 * half)[i];
+        float x[4], p[4], ds[4];
+        f2_unpack(f2_fma(f2_pack(sv[4 * i], sv[4 * i + 1]), c2, f2_pack(nl.x, nl.y)), x[0], x[1]);
+        f2_unpack(f2_fma(f2_pack(sv[4 * i + 2], sv[4 * i + 3]), c2, f2_pack(nl.z, nl.w)), x[2], x[3]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool live = Ls[e] < INFINITY;   // +inf marks a query row without meaning
-          p[e] = live ? ex2(sv[4 * i + e] * scale_log2 - Ls[e]) : 0.f;
-          ds[e] = live ? p[e] * (dpv[4 * i + e] - Ds[e]) : 0.f;
-        }
+        for (int e = 0; e < 4; ++e) p[e] = ex2(x[e]);
+        f2_unpack(f2_mul(f2_pack(p[0], p[1]), f2_add(f2_pack(dpv[4 * i], dpv[4 * i + 1]), f2_pack(nd.x, nd.y))),
+                  ds[0], ds[1]);
+        f2_unpack(f2_mul(f2_pack(p[2], p[3]), f2_add(f2_pack(dpv[4 * i + 2], dpv[4 * i + 3]), f2_pack(nd.z, nd.w))),
+                  ds[2], ds[3]);
         pkp[2 * i] = pack_bf16x2(p[0], p[1]);
         pkp[2 * i + 1] = pack_bf16x2(p[2], p[3]);
         pks[2 * i] = pack_bf16x2(ds[0], ds[1]);

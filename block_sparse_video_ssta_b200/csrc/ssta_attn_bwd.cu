@@ -8,7 +8,9 @@
 // no part (dQ = 0) and pad keys get dK = dV = 0.
 //
 // Kernels, in launch order:
-//   bwd_rowdot_kernel     D per packed row (one warp per row).
+//   bwd_rowdot_kernel     D per packed row (one warp per row); for bf16 also
+//                         -LSE * log2(e) and -D per row of whole tiles, as the
+//                         tensor-core dK/dV kernel reads them.
 //   bwd_transpose_kernel  for each key tile, the ascending list of query tiles
 //                         that keep it (one warp per key tile: a binary search
 //                         in every query tile's sorted list, ballots, prefix).
@@ -88,18 +90,31 @@ __device__ __forceinline__ bool row_valid(const Geom& g, int t, const TileValid&
 
 template <typename T>
 __global__ void __launch_bounds__(kBwdWarps * 32)
-bwd_rowdot_kernel(Geom g, const T* __restrict__ o, const T* __restrict__ dO, float* __restrict__ Dv) {
+bwd_rowdot_kernel(Geom g, const T* __restrict__ o, const T* __restrict__ dO, const float* __restrict__ lse,
+                  float* __restrict__ Dv, float* __restrict__ nl2, float* __restrict__ nd) {
   const int lane = threadIdx.x & 31;
-  const int64_t w = (int64_t)blockIdx.x * kBwdWarps + (threadIdx.x >> 5);   // bh * Lq + row
-  if (w >= (int64_t)g.B * g.H * g.Lq) return;
-  const int64_t row = w % g.Lq;
+  const int64_t Lp = (int64_t)g.NQ * g.N;   // whole tiles: the last text tile's tail rows too
+  const int64_t w = (int64_t)blockIdx.x * kBwdWarps + (threadIdx.x >> 5);   // bh * Lp + row
+  if (w >= (int64_t)g.B * g.H * Lp) return;
+  const int64_t bh = w / Lp, row = w - bh * Lp;
   const int t = (int)(row / g.N);
+  const bool valid = row < g.Lq && row_valid(g, t, tile_valid(g, t), (int)(row - (int64_t)t * g.N));
+  const int64_t wq = bh * g.Lq + row;
   float d = 0.f, unused = 0.f;
-  if (row_valid(g, t, tile_valid(g, t), (int)(row - (int64_t)t * g.N))) {
-    d = dot4(load4(o, w, lane), load4(dO, w, lane));
+  if (valid) {
+    d = dot4(load4(o, wq, lane), load4(dO, wq, lane));
     warp_sum2(d, unused);
   }
-  if (lane == 0) Dv[w] = d;
+  if (lane == 0) {
+    if (row < g.Lq) Dv[wq] = d;
+    if (nl2 != nullptr) {
+      // the tensor-core dK/dV kernel adds these: -LSE in log2 units (-inf for a row that
+      // takes no part, whose P is then exactly 0) and -D
+      const float L = valid ? lse[wq] : -INFINITY;
+      nl2[w] = L > -INFINITY ? -(L * 1.4426950408889634f) : -INFINITY;
+      nd[w] = L > -INFINITY ? -d : 0.f;
+    }
+  }
 }
 
 // For key tile j of head bh: tidx[bh][j][0..tcnt) = query tiles i (ascending) whose
@@ -234,6 +249,9 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
                              void* dq, void* dk, void* dv, const BwdWorkspace& ws, uint8_t* base, cudaStream_t s) {
   const int64_t rows = (int64_t)g.B * g.H * g.Lq, tiles = (int64_t)g.B * g.H * g.NQ;
   float* Dv = reinterpret_cast<float*>(base + ws.rowdot);
+  float* nl2 = kTensorCores<T> ? reinterpret_cast<float*>(base + ws.nl2) : nullptr;
+  float* nd = kTensorCores<T> ? reinterpret_cast<float*>(base + ws.nd) : nullptr;
+  const int64_t prows = (int64_t)g.B * g.H * g.NQ * g.N;
   int32_t* tidx = reinterpret_cast<int32_t*>(base + ws.tidx);
   int32_t* tcnt = reinterpret_cast<int32_t*>(base + ws.tcnt);
   int32_t* status = reinterpret_cast<int32_t*>(base + ws.status);
@@ -242,12 +260,13 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
   const T* tk = static_cast<const T*>(k);
   const T* tv = static_cast<const T*>(v);
   const T* tO = static_cast<const T*>(dO);
-  bwd_rowdot_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, static_cast<const T*>(o), tO, Dv);
+  const unsigned pb = (unsigned)((prows + kBwdWarps - 1) / kBwdWarps);
+  bwd_rowdot_kernel<T><<<pb, kBwdWarps * 32, 0, s>>>(g, static_cast<const T*>(o), tO, lse, Dv, nl2, nd);
   bwd_transpose_kernel<<<tb, kBwdWarps * 32, 0, s>>>(g, kv_idx, kv_cnt, tidx, tcnt, status);
   if constexpr (kTensorCores<T>) {   // bf16: the API guarantees N % 128 == 0
     cudaError_t e = launch_attention_bwd_dq_tc(g, q, k, v, dO, lse, Dv, kv_idx, kv_cnt, dq, status, s);
     if (e != cudaSuccess) return e;
-    e = launch_attention_bwd_dkdv_tc(g, q, k, v, dO, lse, Dv, tidx, tcnt, dk, dv, status, s);
+    e = launch_attention_bwd_dkdv_tc(g, q, k, v, dO, nl2, nd, tidx, tcnt, dk, dv, status, s);
     if (e != cudaSuccess) return e;
   } else {
     bwd_dq_kernel<T><<<rb, kBwdWarps * 32, 0, s>>>(g, tq, tk, tv, tO, lse, Dv, kv_idx, kv_cnt, static_cast<T*>(dq),
@@ -266,7 +285,9 @@ BwdWorkspace bwd_workspace_layout(const Geom& g) {
   BwdWorkspace w{};
   w.status = 0;
   w.rowdot = 256;
-  w.tcnt = w.rowdot + up(bh * (size_t)g.Lq * sizeof(float));
+  w.nl2 = w.rowdot + up(bh * (size_t)g.Lq * sizeof(float));
+  w.nd = w.nl2 + up(bh * (size_t)g.NQ * g.N * sizeof(float));
+  w.tcnt = w.nd + up(bh * (size_t)g.NQ * g.N * sizeof(float));
   w.tidx = w.tcnt + up(bh * (size_t)g.NQ * sizeof(int32_t));
   w.total = w.tidx + up(bh * (size_t)g.NQ * g.NQ * sizeof(int32_t));
   return w;

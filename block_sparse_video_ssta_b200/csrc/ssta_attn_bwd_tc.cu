@@ -348,17 +348,24 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
 // 128-key block, summed over the 128-row query chunks of every query tile that
 // keeps the block's tile (the transposed kept lists).  Warp roles:
 //   warps 0-7  elementwise: warp w serves key rows 32 (w mod 4) .. +31 and query
-//              columns 64 (w / 4) .. +63 of each step: P^T and dS^T from S^T and
-//              dP^T in tensor memory (the per-query LSE and D come from shared
-//              memory); P^T (bf16) over S^T, dS^T (bf16) over dP^T; epilogue
-//              (the warps of query half 0 write dV, those of half 1 dK)
-//   warp  8    producer: K and V of the block once; per step Q and dO by TMA and
-//              the step's LSE (log2 units, +inf for rows without meaning) and D,
-//              loaded and stored to shared memory by the warp's 32 lanes
-//   warp  9    TMEM allocator and MMA issuer: per step dV, dK of the previous
-//              step (A from tensor memory, B = dO and Q read MN-major), then
-//              S^T = K Q^T and dP^T = V dO^T
-// Tensor memory: S^T | dP^T | dV | dK, 128 columns each.
+//              columns 64 (w / 4) .. +63 of each step, in two phases: P^T from
+//              S^T (bf16, written over the S^T columns the warp read), then dS^T
+//              from dP^T and P (bf16, likewise over dP^T); the per-query -LSE (log2 units) and -D come from the
+//              rows the row-dot kernel wrote; epilogue (the warps of query half 0
+//              write dV, those of half 1 dK)
+//   warp  8    producer: K and V of the block once; per step Q (3-stage ring)
+//              and dO (2-stage ring) by TMA, and an L1 prefetch of the step's
+//              -LSE and -D rows
+//   warp  9    TMEM allocator and MMA issuer, in the order
+//                dV(s) += P^T(s) dO(s),  S^T(s+1) = K Q(s+1)^T,
+//                dK(s) += dS^T(s) Q(s),  dP^T(s+1) = V dO(s+1)^T,
+//              so the tensor cores run dV(s) and S^T(s+1) while the elementwise
+//              warps form dS^T(s), and dK(s) and dP^T(s+1) while they take the
+//              exponentials of step s+1.  A product that writes tensor-memory
+//              columns is issued after the one that reads them (one CTA's
+//              products run in issue order): S^T(s+1) after dV(s) reads P^T(s),
+//              dP^T(s+1) after dK(s) reads dS^T(s).
+// Tensor memory: S^T / P^T | dP^T / dS^T | dV | dK, 128 columns each.
 // ============================================================================
 namespace {
 
@@ -368,18 +375,33 @@ using namespace tc;
 constexpr int kKvThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kQStages = 3;   // Q is read by S^T(s) and, a step later, by dK(s)
+constexpr int kOStages = 2;
 constexpr uint32_t kKvOffK = 0;
 constexpr uint32_t kKvOffV = kTileBytes;
-constexpr uint32_t kKvStageBytes = 2 * kTileBytes + 1024;   // Q | dO | L2[128] | D[128]
-constexpr uint32_t kKvOffStage = 2 * kTileBytes;
-constexpr uint32_t kKvOffBar = kKvOffStage + 2 * kKvStageBytes;
-constexpr int kKvNumBars = 10;
+constexpr uint32_t kKvOffQ = 2 * kTileBytes;
+constexpr uint32_t kKvOffO = kKvOffQ + kQStages * kTileBytes;
+constexpr uint32_t kKvOffBar = kKvOffO + kOStages * kTileBytes;
+constexpr int kKvNumBars = 17;
 constexpr uint32_t kKvOffMisc = kKvOffBar + kKvNumBars * 8;
 constexpr uint32_t kKvSmemAlloc = kKvOffMisc + 64 + 1024;
+static_assert(kKvSmemAlloc <= 227 * 1024, "shared memory");
 
 enum : int {
-  KB_KV = 0, KB_QFULL = 1, KB_QEMPTY = 3, KB_SFULL = 5, KB_PREADY = 6, KB_DONE = 7, KB_DRAIN = 8
+  KB_KV = 0, KB_QFULL = 1, KB_QEMPTY = 4, KB_OFULL = 7, KB_OEMPTY = 9, KB_SFULL = 11, KB_PREADY = 12,
+  KB_DPFULL = 13, KB_DSREADY = 14, KB_DONE = 15, KB_DRAIN = 16
 };
+
+// P^T and dS^T are written back in bf16 pairs over the fp32 columns each warp read:
+// query columns 64h .. 64h+63 of S^T (or dP^T) hold, packed, in tensor-memory
+// columns 64h .. 64h+31.  (Packing both halves into columns 0 .. 63 would let the
+// warp of half 1 overwrite fp32 values the warp of half 0 has not loaded yet.)
+// Column of the bf16 A operand for query columns 16 kk .. 16 kk + 15:
+__device__ __forceinline__ uint32_t pcol(int kk) { return 8u * (uint32_t)kk + ((uint32_t)(kk >> 2) << 5); }
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
 
 // Calls f(step, t, ch) for every 128-row chunk with a valid row of every query tile
 // in the transposed list, in list order; stops early when f returns false.
@@ -405,15 +427,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO, const Geom g,
                    const __grid_constant__ ChunkTables tb, const int32_t* __restrict__ tidx, const int32_t* __restrict__ tcnt,
-                   const float* __restrict__ lse, const float* __restrict__ Dv, __nv_bfloat16* __restrict__ dk,
+                   const float* __restrict__ nl2, const float* __restrict__ nd, __nv_bfloat16* __restrict__ dk,
                    __nv_bfloat16* __restrict__ dv, int32_t* __restrict__ status, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
   const uint32_t sK = base + kKvOffK, sV = base + kKvOffV;
-  auto stage = [&](int s) { return base + kKvOffStage + (uint32_t)s * kKvStageBytes; };
-  auto stage_ptr = [&](int s) { return base_ptr + kKvOffStage + (size_t)s * kKvStageBytes; };
+  auto sQ = [&](int i) { return base + kKvOffQ + (uint32_t)i * kTileBytes; };
+  auto sO = [&](int i) { return base + kKvOffO + (uint32_t)i * kTileBytes; };
   auto bar = [&](int i) { return base + kKvOffBar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kKvOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kKvOffMisc + 8);
@@ -449,15 +471,23 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tcount = tcount < 0 ? 0 : g.NQ;
   }
   const int32_t* tlist = tidx + trow * g.NQ;
+  // per-query rows of -LSE and -D: whole tiles per head
+  const int64_t Lp = (int64_t)g.NQ * g.N;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(KB_KV), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(KB_QFULL + s), 33);      // the TMA transaction arrival + 32 producer lanes
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(bar(KB_QFULL + s), 1);
       mbar_init(bar(KB_QEMPTY + s), 1);
+    }
+    for (int s = 0; s < kOStages; ++s) {
+      mbar_init(bar(KB_OFULL + s), 1);
+      mbar_init(bar(KB_OEMPTY + s), 1);
     }
     mbar_init(bar(KB_SFULL), 1);
     mbar_init(bar(KB_PREADY), 256);
+    mbar_init(bar(KB_DPFULL), 1);
+    mbar_init(bar(KB_DSREADY), 256);
     mbar_init(bar(KB_DONE), 1);
     mbar_init(bar(KB_DRAIN), 1);
     *abort_flag = 0;
@@ -484,91 +514,100 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
-    const int z = (int)bh;
     if (lane == 0) {
+      const int z = (int)bh;
       mbar_expect_tx(bar(KB_KV), 2 * kTileBytes);
       for (int b = 0; b < 2; ++b) {
         tma_load_3d(sK + b * kBox, &tmK, b * 64, krow0, z, bar(KB_KV));
         tma_load_3d(sV + b * kBox, &tmV, b * 64, krow0, z, bar(KB_KV));
       }
-    }
-    int issued[2] = {0, 0};
-    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int t, int ch) -> bool {
-      const int s = step & 1;
-      const uint32_t ph = (uint32_t)((step >> 1) & 1);
-      if (!wait_warp(bar(KB_QEMPTY + s), ph ^ 1u, ctl)) return false;
-      const int qrow = t * g.N + ch * kChunk;
-      if (lane == 0) {
-        mbar_expect_tx(bar(KB_QFULL + s), 2 * kTileBytes);
-        for (int b = 0; b < 2; ++b) {
-          tma_load_3d(stage(s) + b * kBox, &tmQ, b * 64, qrow, z, bar(KB_QFULL + s));
-          tma_load_3d(stage(s) + kTileBytes + b * kBox, &tmDO, b * 64, qrow, z, bar(KB_QFULL + s));
-        }
-      }
-      float* l2 = reinterpret_cast<float*>(stage_ptr(s) + 2 * kTileBytes);
-      float* dd = l2 + 128;
+      int nq[kQStages] = {0, 0, 0}, no[kOStages] = {0, 0};
+      const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int t, int ch) -> bool {
+        const int qs = step % kQStages, os = step & 1;
+        const int qrow = t * g.N + ch * kChunk;
+        if (!wait_bounded(bar(KB_QEMPTY + qs), (uint32_t)(((step / kQStages) & 1) ^ 1), ctl)) return false;
+        mbar_expect_tx(bar(KB_QFULL + qs), kTileBytes);
+        for (int b = 0; b < 2; ++b) tma_load_3d(sQ(qs) + b * kBox, &tmQ, b * 64, qrow, z, bar(KB_QFULL + qs));
+        ++nq[qs];
+        if (!wait_bounded(bar(KB_OEMPTY + os), (uint32_t)(((step >> 1) & 1) ^ 1), ctl)) return false;
+        mbar_expect_tx(bar(KB_OFULL + os), kTileBytes);
+        for (int b = 0; b < 2; ++b) tma_load_3d(sO(os) + b * kBox, &tmDO, b * 64, qrow, z, bar(KB_OFULL + os));
+        ++no[os];
+        // the step's 128 values of -LSE and of -D (four 128-byte lines each) into L1
+        const float* pl = nl2 + bh * Lp + qrow;
+        const float* pd = nd + bh * Lp + qrow;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = lane + 32 * i;
-        const int64_t row = (int64_t)qrow + c;
-        const bool ok = row < g.Lq && key_valid(g, tb, t, ch * kChunk + c);
-        const float L = ok ? __ldg(lse + bh * g.Lq + row) : -INFINITY;
-        // negated, so the elementwise step adds them: -LSE in log2 units (-inf for a row without
-        // meaning, whose P is then exactly 0) and -D
-        l2[c] = L > -INFINITY ? -(L * 1.4426950408889634f) : -INFINITY;
-        dd[c] = L > -INFINITY ? -__ldg(Dv + bh * g.Lq + row) : 0.f;
+        for (int i = 0; i < 4; ++i) {
+          prefetch_l1(pl + 32 * i);
+          prefetch_l1(pd + 32 * i);
+        }
+        return true;
+      });
+      if (n < 0) {
+        drain_wait(bar(KB_KV), 0, kTimeoutNs);
+        for (int s = 0; s < kQStages; ++s)
+          if (nq[s] > 0) drain_wait(bar(KB_QFULL + s), (uint32_t)((nq[s] - 1) & 1), kTimeoutNs);
+        for (int s = 0; s < kOStages; ++s)
+          if (no[s] > 0) drain_wait(bar(KB_OFULL + s), (uint32_t)((no[s] - 1) & 1), kTimeoutNs);
       }
-      mbar_arrive(bar(KB_QFULL + s));
-      ++issued[s];
-      return true;
-    });
-    if (n < 0 && lane == 0) {
-      drain_wait(bar(KB_KV), 0, kTimeoutNs);
-      for (int s = 0; s < 2; ++s)
-        if (issued[s] > 0) drain_wait(bar(KB_QFULL + s), (uint32_t)((issued[s] - 1) & 1), kTimeoutNs);
+      if (n >= 0 && tcount == 0) drain_wait(bar(KB_KV), 0, kTimeoutNs);
     }
-    if (n >= 0 && lane == 0 && tcount == 0) drain_wait(bar(KB_KV), 0, kTimeoutNs);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const bool ok = wait_bounded(bar(KB_KV), 0, ctl);
-      auto grad_step = [&](int sp) -> bool {   // dV, dK of step sp
-        if (!wait_bounded(bar(KB_PREADY), (uint32_t)(sp & 1), ctl)) return false;
+      auto s_step = [&](int s) -> bool {   // S^T(s) = K Q(s)^T
+        if (!wait_bounded(bar(KB_QFULL + s % kQStages), (uint32_t)((s / kQStages) & 1), ctl)) return false;
         tc_fence_after();
-        const uint32_t qb = stage(sp & 1), ob = qb + kTileBytes;
+        const uint32_t qb = sQ(s % kQStages);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+          mma_ss(tS, desc_kmajor(sK + off), desc_kmajor(qb + off), kIdescKK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(KB_SFULL));
+        return true;
+      };
+      auto dp_step = [&](int s) -> bool {   // dP^T(s) = V dO(s)^T
+        if (!wait_bounded(bar(KB_OFULL + (s & 1)), (uint32_t)((s >> 1) & 1), ctl)) return false;
+        tc_fence_after();
+        const uint32_t ob = sO(s & 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
+          mma_ss(tP, desc_kmajor(sV + off), desc_kmajor(ob + off), kIdescKK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(KB_DPFULL));
+        return true;
+      };
+      auto dv_step = [&](int s) -> bool {   // dV += P^T(s) dO(s): A = P^T in tensor memory, B = dO MN-major
+        if (!wait_bounded(bar(KB_PREADY), (uint32_t)(s & 1), ctl)) return false;
+        tc_fence_after();
+        const uint32_t ob = sO(s & 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDV, tS + 8u * kk, desc_mnmajor(ob + 2048u * kk), kIdescKMN, (sp > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tDV, tS + pcol(kk), desc_mnmajor(ob + 2048u * kk), kIdescKMN, (s > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(KB_OEMPTY + (s & 1)));
+        return true;
+      };
+      auto dk_step = [&](int s) -> bool {   // dK += dS^T(s) Q(s): A = dS^T in tensor memory, B = Q MN-major
+        if (!wait_bounded(bar(KB_DSREADY), (uint32_t)(s & 1), ctl)) return false;
+        tc_fence_after();
+        const uint32_t qb = sQ(s % kQStages);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDK, tP + 8u * kk, desc_mnmajor(qb + 2048u * kk), kIdescKMN, (sp > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(KB_DONE));
-        tc_commit(bar(KB_QEMPTY + (sp & 1)));
+          mma_ts(tDK, tP + pcol(kk), desc_mnmajor(qb + 2048u * kk), kIdescKMN, (s > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(KB_QEMPTY + s % kQStages));
         return true;
       };
       int n = -1;
       if (ok) {
         n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
-          const int s = step & 1;
-          if (step > 0 && !grad_step(step - 1)) return false;
-          if (!wait_bounded(bar(KB_QFULL + s), (uint32_t)((step >> 1) & 1), ctl)) return false;
-          tc_fence_after();
-          const uint32_t qb = stage(s), ob = qb + kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tS, desc_kmajor(sK + off), desc_kmajor(qb + off), kIdescKK, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tP, desc_kmajor(sV + off), desc_kmajor(ob + off), kIdescKK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(KB_SFULL));
-          return true;
+          if (step == 0) return s_step(0) && dp_step(0);
+          return dv_step(step - 1) && s_step(step) && dk_step(step - 1) && dp_step(step);
         });
       }
-      if (n > 0) grad_step(n - 1);
+      if (n > 0 && dv_step(n - 1) && dk_step(n - 1)) tc_commit(bar(KB_DONE));
       tc_commit(bar(KB_DRAIN));
       drain_wait(bar(KB_DRAIN), 0, kTimeoutNs);
     }
@@ -579,48 +618,61 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
     const int64_t row = (int64_t)krow0 + grp * 32 + lane;
     const bool key_ok = row < g.Lq && key_valid(g, tb, kt, (int)(row - (int64_t)kt * g.N));
-    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
+    const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+    const float* nl_head = nl2 + bh * Lp + 64 * half;
+    const float* nd_head = nd + bh * Lp + 64 * half;
+    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int t, int ch) -> bool {
+      const int64_t qrow = (int64_t)t * g.N + ch * kChunk;
+      const float4* nlv = reinterpret_cast<const float4*>(nl_head + qrow);
+      const float4* ndv = reinterpret_cast<const float4*>(nd_head + qrow);
+      // P^T = 2^(S^T * scale - LSE), two query columns per f32x2 instruction (-LSE is -inf
+      // for a query row without meaning: P = 0); kept in fp32 for dS, written over S^T in bf16
       if (!wait_warp(bar(KB_SFULL), (uint32_t)(step & 1), ctl)) return false;
-      // the producer's per-query values of this stage: acquire them from its own barrier
-      if (!wait_warp(bar(KB_QFULL + (step & 1)), (uint32_t)((step >> 1) & 1), ctl)) return false;
       tc_fence_after();
-      const float* l2 = reinterpret_cast<const float*>(stage_ptr(step & 1) + 2 * kTileBytes);
-      const float* dd = l2 + 128;
-      float sv[64], dpv[64];
-      tmem_ld64(tS + lane_off + 64u * half, sv);
-      tmem_ld64(tP + lane_off + 64u * half, dpv);
-      // P = 2^(s * scale - LSE), dS = P (dP - D), two query columns per f32x2 instruction; the
-      // stage holds -LSE (log2 units, -inf for a row without meaning: P = 0) and -D
-      const uint64_t c2 = f2_pack(scale_log2, scale_log2);
-      uint32_t pkp[32], pks[32];
+      float pv[64];
+      tmem_ld64(tS + lane_off + 64u * half, pv);
+      uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float4 nl = reinterpret_cast<const float4*>(l2 + 64 * half)[i];
-        const float4 nd = reinterpret_cast<const float4*>(dd + 64 * half)[i];
-        float x[4], p[4], ds[4];
-        f2_unpack(f2_fma(f2_pack(sv[4 * i], sv[4 * i + 1]), c2, f2_pack(nl.x, nl.y)), x[0], x[1]);
-        f2_unpack(f2_fma(f2_pack(sv[4 * i + 2], sv[4 * i + 3]), c2, f2_pack(nl.z, nl.w)), x[2], x[3]);
+        const float4 nl = __ldg(nlv + i);
+        float x[4];
+        f2_unpack(f2_fma(f2_pack(pv[4 * i], pv[4 * i + 1]), c2, f2_pack(nl.x, nl.y)), x[0], x[1]);
+        f2_unpack(f2_fma(f2_pack(pv[4 * i + 2], pv[4 * i + 3]), c2, f2_pack(nl.z, nl.w)), x[2], x[3]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) p[e] = ex2(x[e]);
-        f2_unpack(f2_mul(f2_pack(p[0], p[1]), f2_add(f2_pack(dpv[4 * i], dpv[4 * i + 1]), f2_pack(nd.x, nd.y))),
-                  ds[0], ds[1]);
-        f2_unpack(f2_mul(f2_pack(p[2], p[3]), f2_add(f2_pack(dpv[4 * i + 2], dpv[4 * i + 3]), f2_pack(nd.z, nd.w))),
-                  ds[2], ds[3]);
-        pkp[2 * i] = pack_bf16x2(p[0], p[1]);
-        pkp[2 * i + 1] = pack_bf16x2(p[2], p[3]);
-        pks[2 * i] = pack_bf16x2(ds[0], ds[1]);
-        pks[2 * i + 1] = pack_bf16x2(ds[2], ds[3]);
+        for (int e = 0; e < 4; ++e) pv[4 * i + e] = ex2(x[e]);
+        pk[2 * i] = pack_bf16x2(pv[4 * i], pv[4 * i + 1]);
+        pk[2 * i + 1] = pack_bf16x2(pv[4 * i + 2], pv[4 * i + 3]);
       }
-      tmem_st32u(tS + lane_off + 32u * half, pkp);
-      tmem_st32u(tP + lane_off + 32u * half, pks);
+      tmem_st32u(tS + lane_off + 64u * half, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(KB_PREADY));
+      // dS^T = P^T (dP^T - D), written over dP^T in bf16
+      if (!wait_warp(bar(KB_DPFULL), (uint32_t)(step & 1), ctl)) return false;
+      tc_fence_after();
+      float dpv[64];
+      tmem_ld64(tP + lane_off + 64u * half, dpv);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float4 d4 = __ldg(ndv + i);
+        float ds[4];
+        f2_unpack(f2_mul(f2_pack(pv[4 * i], pv[4 * i + 1]), f2_add(f2_pack(dpv[4 * i], dpv[4 * i + 1]), f2_pack(d4.x, d4.y))),
+                  ds[0], ds[1]);
+        f2_unpack(f2_mul(f2_pack(pv[4 * i + 2], pv[4 * i + 3]),
+                         f2_add(f2_pack(dpv[4 * i + 2], dpv[4 * i + 3]), f2_pack(d4.z, d4.w))),
+                  ds[2], ds[3]);
+        pk[2 * i] = pack_bf16x2(ds[0], ds[1]);
+        pk[2 * i + 1] = pack_bf16x2(ds[2], ds[3]);
+      }
+      tmem_st32u(tP + lane_off + 64u * half, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(KB_DSREADY));
       return true;
     });
     // epilogue: the warps of column half 0 write dV, those of half 1 write dK
     bool have = n > 0;
-    if (have) have = wait_warp(bar(KB_DONE), (uint32_t)((n - 1) & 1), ctl);
+    if (have) have = wait_warp(bar(KB_DONE), 0u, ctl);
     tc_fence_after();
     const bool write = row < g.Lq && !*abort_flag;
     const float sc = scale_log2 * 0.69314718055994531f;
@@ -663,7 +715,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 }  // namespace
 
 cudaError_t launch_attention_bwd_dkdv_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
-                                         const float* lse, const float* Dv, const int32_t* tidx,
+                                         const float* nl2, const float* nd, const int32_t* tidx,
                                          const int32_t* tcnt, void* dk, void* dv, int32_t* status, cudaStream_t s) {
   const int64_t BH = (int64_t)g.B * g.H;
   if (BH == 0) return cudaSuccess;
@@ -682,7 +734,7 @@ cudaError_t launch_attention_bwd_dkdv_tc(const Geom& g, const void* q, const voi
   }
   const int64_t units = BH * (int64_t)g.NQ * (g.N / 128);
   bwd_dkdv_tc_kernel<<<(unsigned)units, kKvThreads, kKvSmemAlloc, s>>>(
-      mq, mk, mv, mdo, g, make_chunk_tables(g), tidx, tcnt, lse, Dv, static_cast<__nv_bfloat16*>(dk),
+      mq, mk, mv, mdo, g, make_chunk_tables(g), tidx, tcnt, nl2, nd, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv), status, g.scale * 1.4426950408889634f);
   return cudaGetLastError();
 }

@@ -61,6 +61,8 @@ struct ImportanceBufs {
 struct BwdWorkspace {
   size_t status;   // int32 device status word
   size_t rowdot;   // fp32 [BH, Lq], D = rowsum(dO * O)
+  size_t nl2;      // fp32 [BH, NQ * N], -LSE * log2(e) per packed row (-inf: pad row or no kept key)
+  size_t nd;       // fp32 [BH, NQ * N], -D per packed row (0 where nl2 is -inf)
   size_t tcnt;     // int32 [BH, NQ], query tiles keeping each key tile
   size_t tidx;     // int32 [BH, NQ, NQ], those query tiles, ascending
   size_t total;
@@ -99,7 +101,7 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
                                        const int32_t* kv_cnt, void* dq, int32_t* status, cudaStream_t s);
 // bf16, N % 128 == 0: dK and dV on the tensor cores (tidx/tcnt: the transposed lists).
 cudaError_t launch_attention_bwd_dkdv_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
-                                         const float* lse, const float* Dv, const int32_t* tidx,
+                                         const float* nl2, const float* nd, const int32_t* tidx,
                                          const int32_t* tcnt, void* dk, void* dv, int32_t* status, cudaStream_t s);
 cudaError_t launch_attention_bf16_tc(const Geom& g, const void* qp, const void* kp, const void* vp,
                                      const int32_t* kv_idx, const int32_t* kv_cnt, void* o, float* lse,

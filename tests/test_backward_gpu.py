@@ -6,7 +6,11 @@ Tolerances, from the arithmetic: fp32 keeps fp32 end to end (sums over a few
 thousand keys): relative L2 and max-abs (scaled by the largest reference value)
 1e-4.  bf16 stores O and the three gradients in bf16 (2^-9 relative per element)
 and D = rowsum(dO * O) is formed from the stored O: relative L2 1e-2, max-abs
-2e-2 of the largest reference value."""
+2e-2 of the largest reference value.  Each output row is also held to its own
+relative L2 error (rows above 1e-3 of the largest row norm): 1e-4 for fp32, 5e-2
+for bf16 (P and dS enter the products rounded to bf16, 2^-9 relative each, and the
+row is stored in bf16), so that a fault confined to a few rows cannot hide inside
+the whole-tensor figures."""
 import numpy as np
 import pytest
 import torch
@@ -19,7 +23,7 @@ from ssta_parity import compare_masks, gpu_kept, oracle_mask, run_gpu, to_np
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"f32": dict(rel=1e-4, mx=1e-4), "bf16": dict(rel=1e-2, mx=2e-2)}
+TOL = {"f32": dict(rel=1e-4, mx=1e-4, row=1e-4), "bf16": dict(rel=1e-2, mx=2e-2, row=5e-2)}
 
 
 def _oracle_packed(w, x, heads=None):
@@ -57,9 +61,16 @@ def _check(w, seed=0):
         scale = max(np.abs(want).max(), 1e-30)
         mx = float(np.abs(a - want).max()) / scale
         rel = float(np.linalg.norm(a - want) / max(np.linalg.norm(want), 1e-30))
-        stats[name] = (mx, rel)
+        # worst relative L2 error of one row, over rows above 1e-3 of the largest row norm
+        rn = np.linalg.norm(want.reshape(-1, want.shape[-1]), axis=1)
+        en = np.linalg.norm((a - want).reshape(-1, want.shape[-1]), axis=1)
+        big = rn > 1e-3 * max(rn.max(), 1e-30)
+        row_rel = float((en[big] / rn[big]).max()) if big.any() else 0.0
+        stats[name] = (mx, rel, row_rel)
         assert mx <= TOL[w.dtype]["mx"] and rel <= TOL[w.dtype]["rel"], (name, mx, rel)
-    print(f"\n[bwd {w.name} {w.dtype}] " + " ".join(f"{k}: max {v[0]:.2e} rel {v[1]:.2e}" for k, v in stats.items()))
+        assert row_rel <= TOL[w.dtype]["row"], (name, row_rel)
+    print(f"\n[bwd {w.name} {w.dtype}] " + " ".join(f"{k}: max {v[0]:.2e} rel {v[1]:.2e} row {v[2]:.2e}"
+                                                    for k, v in stats.items()))
     return stats
 
 
@@ -122,3 +133,27 @@ def test_backward_full_size_sampled(cuda_ok):
         stats[name] = (mx, rel, int(rows.sum()))
         assert mx <= TOL["bf16"]["mx"] and rel <= TOL["bf16"]["rel"], (name, mx, rel)
     print("\n[bwd 720p-10s sampled] " + " ".join(f"{k}: max {v[0]:.2e} rel {v[1]:.2e} rows {v[2]}" for k, v in stats.items()))
+
+
+def test_backward_full_size_deterministic(cuda_ok):
+    """Three backward calls on the same 720p-10s inputs (as bench.py times it) give the
+    same bytes: every sum runs in a fixed order, and no warp may read tensor memory that
+    another warp of its lane group has already overwritten (a race there changes a few
+    percent of the dK and dV rows from call to call while staying inside the loose
+    whole-tensor tolerances above)."""
+    w = si.get_workload("p720_10s_bf16")
+    x = si.make_inputs(w, 0, device="cuda")
+    r = run_gpu(w, x, want_scores=False)
+    del x
+    d = S.desc_from(w)
+    dO = torch.randn(r["O_packed"].shape, device="cuda", generator=torch.Generator(device="cuda").manual_seed(5)
+                     ).to(r["O_packed"].dtype)
+    first = None
+    for _ in range(3):
+        out = S.ssta_attention_bwd(d, r["qp"], r["kp"], r["vp"], r["O_packed"], r["LSE"], dO, r["kv_idx"], r["kv_cnt"])
+        assert S.ssta_read_device_status(out[3]) == 0
+        if first is None:
+            first = [t.clone() for t in out[:3]]
+            continue
+        for name, a, b in zip(("dq", "dk", "dv"), first, out[:3]):
+            assert torch.equal(a, b), (name, int((a != b).sum()))

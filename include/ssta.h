@@ -196,8 +196,9 @@ ssta_status ssta_attention_fwd(const ssta_desc* desc, const void* q_packed, cons
  *   q/k/v/o/do_packed [B,H,Lq,D] (read; o and lse as ssta_attention_fwd wrote them,
  *   do = dL/dO), kv_idx/kv_cnt as ssta_build_block_mask wrote them (ascending lists
  *   required), dq/dk/dv_packed [B,H,Lq,D] (written in full), all of `dtype`;
- *   workspace >= info.bwd_workspace_bytes (status word, per-row D, and for every key
- *   tile the list of query tiles keeping it).
+ *   workspace >= info.bwd_workspace_bytes (status word, per-row D, per-row -LSE and -D
+ *   over whole tiles for the bf16 kernels, and for every key tile the list of query
+ *   tiles keeping it).
  * bf16 (N % 128 == 0 required, as for ssta_attention_fwd): tcgen05 tensor-core
  * kernels, one for dQ over each query tile's kept list, one for dK and dV over the
  * query tiles keeping each key tile.  fp32: SIMT kernels with fp32 arithmetic.

@@ -350,12 +350,14 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
 //   warps 0-7  elementwise: warp w serves key rows 32 (w mod 4) .. +31 and query
 //              columns 64 (w / 4) .. +63 of each step, in two phases: P^T from
 //              S^T (bf16, written over the S^T columns the warp read), then dS^T
-//              from dP^T and P (bf16, likewise over dP^T); the per-query -LSE (log2 units) and -D come from the
-//              rows the row-dot kernel wrote; epilogue (the warps of query half 0
+//              from dP^T and P (bf16, likewise over dP^T); the per-query -LSE
+//              (log2 units) and -D are the rows the row-dot kernel wrote, staged
+//              in shared memory with dO; epilogue (the warps of query half 0
 //              write dV, those of half 1 dK)
 //   warp  8    producer: K and V of the block once; per step Q (3-stage ring)
-//              and dO (2-stage ring) by TMA, and an L1 prefetch of the step's
-//              -LSE and -D rows
+//              by TMA, and dO (2-stage ring) by TMA with the step's -LSE and -D
+//              rows by bulk copy onto the same barrier (the dO stage is released
+//              after dK(s), when the elementwise step has read them)
 //   warp  9    TMEM allocator and MMA issuer, in the order
 //                dV(s) += P^T(s) dO(s),  S^T(s+1) = K Q(s+1)^T,
 //                dK(s) += dS^T(s) Q(s),  dP^T(s+1) = V dO(s+1)^T,
@@ -381,11 +383,19 @@ constexpr uint32_t kKvOffK = 0;
 constexpr uint32_t kKvOffV = kTileBytes;
 constexpr uint32_t kKvOffQ = 2 * kTileBytes;
 constexpr uint32_t kKvOffO = kKvOffQ + kQStages * kTileBytes;
-constexpr uint32_t kKvOffBar = kKvOffO + kOStages * kTileBytes;
+constexpr uint32_t kKvOffLD = kKvOffO + kOStages * kTileBytes;   // per dO stage: -LSE[128] | -D[128]
+constexpr uint32_t kKvLDBytes = 2 * 128 * sizeof(float);
+constexpr uint32_t kKvOffBar = kKvOffLD + kOStages * kKvLDBytes;
 constexpr int kKvNumBars = 17;
 constexpr uint32_t kKvOffMisc = kKvOffBar + kKvNumBars * 8;
-constexpr uint32_t kKvSmemAlloc = kKvOffMisc + 64 + 1024;
-static_assert(kKvSmemAlloc <= 227 * 1024, "shared memory");
+constexpr uint32_t kKvSmemUsed = kKvOffMisc + 64;
+constexpr uint32_t kSmemMax = 227 * 1024;
+// The layout leaves less than 1 KB for aligning the dynamic shared memory base to
+// 1024 bytes (which the 128-byte swizzle needs); the kernel checks the base it got
+// (the runtime places it 1024-aligned when the kernel declares no static shared
+// memory) and reports SSTA_ERR_ALIGNMENT rather than overrun.
+constexpr uint32_t kKvSmemAlloc = kKvSmemUsed + 1024 <= kSmemMax ? kKvSmemUsed + 1024 : kSmemMax;
+static_assert(kKvSmemUsed <= kSmemMax, "shared memory");
 
 enum : int {
   KB_KV = 0, KB_QFULL = 1, KB_QEMPTY = 4, KB_OFULL = 7, KB_OEMPTY = 9, KB_SFULL = 11, KB_PREADY = 12,
@@ -398,10 +408,6 @@ enum : int {
 // warp of half 1 overwrite fp32 values the warp of half 0 has not loaded yet.)
 // Column of the bf16 A operand for query columns 16 kk .. 16 kk + 15:
 __device__ __forceinline__ uint32_t pcol(int kk) { return 8u * (uint32_t)kk + ((uint32_t)(kk >> 2) << 5); }
-
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
-}
 
 // Calls f(step, t, ch) for every 128-row chunk with a valid row of every query tile
 // in the transposed list, in list order; stops early when f returns false.
@@ -436,6 +442,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t sK = base + kKvOffK, sV = base + kKvOffV;
   auto sQ = [&](int i) { return base + kKvOffQ + (uint32_t)i * kTileBytes; };
   auto sO = [&](int i) { return base + kKvOffO + (uint32_t)i * kTileBytes; };
+  auto sLD = [&](int i) { return base + kKvOffLD + (uint32_t)i * kKvLDBytes; };
   auto bar = [&](int i) { return base + kKvOffBar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kKvOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kKvOffMisc + 8);
@@ -443,6 +450,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const Ctl ctl{abort_flag, status, kTimeoutNs};
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (base - raw + kKvSmemUsed > kKvSmemAlloc) {   // uniform over the CTA: nothing started yet
+    if (threadIdx.x == 0) atomicExch(status, (int)SSTA_ERR_ALIGNMENT);
+    return;
+  }
 
   // ---- work unit: one 128-key block of a key tile; text key tiles first (longest lists)
   const int blocks = g.N / 128;
@@ -530,17 +541,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int b = 0; b < 2; ++b) tma_load_3d(sQ(qs) + b * kBox, &tmQ, b * 64, qrow, z, bar(KB_QFULL + qs));
         ++nq[qs];
         if (!wait_bounded(bar(KB_OEMPTY + os), (uint32_t)(((step >> 1) & 1) ^ 1), ctl)) return false;
-        mbar_expect_tx(bar(KB_OFULL + os), kTileBytes);
+        // dO and the step's 128 values of -LSE and of -D, on one barrier
+        mbar_expect_tx(bar(KB_OFULL + os), kTileBytes + kKvLDBytes);
         for (int b = 0; b < 2; ++b) tma_load_3d(sO(os) + b * kBox, &tmDO, b * 64, qrow, z, bar(KB_OFULL + os));
+        bulk_load(sLD(os), nl2 + bh * Lp + qrow, kKvLDBytes / 2, bar(KB_OFULL + os));
+        bulk_load(sLD(os) + kKvLDBytes / 2, nd + bh * Lp + qrow, kKvLDBytes / 2, bar(KB_OFULL + os));
         ++no[os];
-        // the step's 128 values of -LSE and of -D (four 128-byte lines each) into L1
-        const float* pl = nl2 + bh * Lp + qrow;
-        const float* pd = nd + bh * Lp + qrow;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          prefetch_l1(pl + 32 * i);
-          prefetch_l1(pd + 32 * i);
-        }
         return true;
       });
       if (n < 0) {
@@ -587,7 +593,6 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tDV, tS + pcol(kk), desc_mnmajor(ob + 2048u * kk), kIdescKMN, (s > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(KB_OEMPTY + (s & 1)));
         return true;
       };
       auto dk_step = [&](int s) -> bool {   // dK += dS^T(s) Q(s): A = dS^T in tensor memory, B = Q MN-major
@@ -598,6 +603,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tDK, tP + pcol(kk), desc_mnmajor(qb + 2048u * kk), kIdescKMN, (s > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(KB_QEMPTY + s % kQStages));
+        // the dO stage also holds the -LSE and -D the elementwise step read up to DSREADY(s)
+        tc_commit(bar(KB_OEMPTY + (s & 1)));
         return true;
       };
       int n = -1;
@@ -619,14 +626,14 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int64_t row = (int64_t)krow0 + grp * 32 + lane;
     const bool key_ok = row < g.Lq && key_valid(g, tb, kt, (int)(row - (int64_t)kt * g.N));
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
-    const float* nl_head = nl2 + bh * Lp + 64 * half;
-    const float* nd_head = nd + bh * Lp + 64 * half;
-    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int t, int ch) -> bool {
-      const int64_t qrow = (int64_t)t * g.N + ch * kChunk;
-      const float4* nlv = reinterpret_cast<const float4*>(nl_head + qrow);
-      const float4* ndv = reinterpret_cast<const float4*>(nd_head + qrow);
+    const int n = for_each_qchunk(g, tb, tlist, tcount, [&](int step, int, int) -> bool {
+      const float* ld = reinterpret_cast<const float*>(base_ptr + kKvOffLD + (size_t)(step & 1) * kKvLDBytes);
+      const float4* nlv = reinterpret_cast<const float4*>(ld + 64 * half);
+      const float4* ndv = reinterpret_cast<const float4*>(ld + 128 + 64 * half);
       // P^T = 2^(S^T * scale - LSE), two query columns per f32x2 instruction (-LSE is -inf
-      // for a query row without meaning: P = 0); kept in fp32 for dS, written over S^T in bf16
+      // for a query row without meaning: P = 0); kept in fp32 for dS, written over S^T in bf16.
+      // The stage's -LSE and -D arrive with dO: acquire them from its barrier.
+      if (!wait_warp(bar(KB_OFULL + (step & 1)), (uint32_t)((step >> 1) & 1), ctl)) return false;
       if (!wait_warp(bar(KB_SFULL), (uint32_t)(step & 1), ctl)) return false;
       tc_fence_after();
       float pv[64];
@@ -634,7 +641,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float4 nl = __ldg(nlv + i);
+        const float4 nl = nlv[i];
         float x[4];
         f2_unpack(f2_fma(f2_pack(pv[4 * i], pv[4 * i + 1]), c2, f2_pack(nl.x, nl.y)), x[0], x[1]);
         f2_unpack(f2_fma(f2_pack(pv[4 * i + 2], pv[4 * i + 3]), c2, f2_pack(nl.z, nl.w)), x[2], x[3]);
@@ -654,7 +661,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_ld64(tP + lane_off + 64u * half, dpv);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float4 d4 = __ldg(ndv + i);
+        const float4 d4 = ndv[i];
         float ds[4];
         f2_unpack(f2_mul(f2_pack(pv[4 * i], pv[4 * i + 1]), f2_add(f2_pack(dpv[4 * i], dpv[4 * i + 1]), f2_pack(d4.x, d4.y))),
                   ds[0], ds[1]);

@@ -8,14 +8,16 @@
 // in 128-key chunks.  Warp roles:
 //   warps 0-7  elementwise: warp w serves query rows 32 (w mod 4) .. +31 and key
 //              columns 64 (w / 4) .. +63 of each chunk: P and dS from S and dP in
-//              tensor memory, dS (bf16) into shared memory; epilogue dQ * scale
-//   warp  8    TMA producer: Q and dO once, then K and V chunks (2-stage rings)
+//              tensor memory, dS (bf16) back into tensor memory; epilogue dQ * scale
+//   warp  8    TMA producer: Q and dO once, then K (3-stage ring: K(j) is read by
+//              S(j) and, a chunk later, by dQ) and V (2-stage ring) chunks
 //   warp  9    TMEM allocator and tcgen05.mma issuer
-// Tensor memory: S (fp32, 128 columns), dP (128 columns), dQ accumulator (128).
-// Shared memory: Q, dO, the K and V rings and dS (K-major, 128-byte swizzle).
+// Tensor memory: S (fp32, 128 columns), dP (128), dQ accumulator (128), dS (bf16
+// pairs: key columns 64h .. 64h+63 packed in columns 64h .. 64h+31 of the last 128).
+// Shared memory: Q, dO and the K and V rings (128-byte swizzle).
 // Per chunk j the MMA warp issues S(j) = Q K(j)^T and dP(j) = dO V(j)^T as soon
 // as the elementwise warps have loaded S(j-1) and dP(j-1) into registers, then
-// dQ += dS(j-1) K(j-1) (A = dS from shared memory, B = K read MN-major) once
+// dQ += dS(j-1) K(j-1) (A = dS from tensor memory, B = K read MN-major) once
 // dS(j-1) is written: the next chunk's S and dP run during this chunk's
 // exponentials.  dS is overwritten only after the previous dQ product finished.
 // Every wait is bounded (ssta_wait.cuh), as in the forward kernel.
@@ -35,22 +37,29 @@ constexpr uint64_t kTimeoutNs = 1500000000ull;
 constexpr int kDqThreads = 320;
 constexpr int kDqProducerWarp = 8;
 constexpr int kDqMmaWarp = 9;
-constexpr int kStages = 2;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffDO = kOffQ + kTileBytes;
 constexpr uint32_t kOffK = kOffDO + kTileBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffDS = kOffV + kStages * kTileBytes;   // dS (bf16), K-major, 128-byte swizzle
-constexpr uint32_t kOffBar = kOffDS + kTileBytes;
-constexpr int kNumBars = 14;
+constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
+constexpr int kNumBars = 16;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemAlloc = kOffMisc + 64 + 1024;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 
 enum : int {
-  BAR_Q = 0, BAR_KFULL = 1, BAR_KEMPTY = 3, BAR_VFULL = 5, BAR_VEMPTY = 7,
-  BAR_SFULL = 9, BAR_SFREE = 10, BAR_DSREADY = 11, BAR_DQDONE = 12, BAR_DRAIN = 13
+  BAR_Q = 0, BAR_KFULL = 1, BAR_KEMPTY = 4, BAR_VFULL = 7, BAR_VEMPTY = 9,
+  BAR_SFULL = 11, BAR_SFREE = 12, BAR_DSREADY = 13, BAR_DQDONE = 14, BAR_DRAIN = 15
 };
+
+// dS and P^T are written back in bf16 pairs over (or, for dS in the dQ kernel, beside)
+// fp32 columns each warp read: key (or query) columns 64h .. 64h+63 are packed in
+// tensor-memory columns 64h .. 64h+31 of the region, so the two warps of a lane group
+// never write columns the other one reads.  Column of the bf16 A operand for the 16
+// columns 16 kk .. 16 kk + 15:
+__device__ __forceinline__ uint32_t pcol(int kk) { return 8u * (uint32_t)kk + ((uint32_t)(kk >> 2) << 5); }
 
 __global__ void __launch_bounds__(kDqThreads, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -62,7 +71,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw);
-  const uint32_t sQ = base + kOffQ, sDO = base + kOffDO, sK = base + kOffK, sV = base + kOffV, sDS = base + kOffDS;
+  const uint32_t sQ = base + kOffQ, sDO = base + kOffDO, sK = base + kOffK, sV = base + kOffV;
   auto bar = [&](int i) { return base + kOffBar + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffMisc + 8);
@@ -100,9 +109,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(BAR_KFULL + s), 1);
       mbar_init(bar(BAR_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(bar(BAR_VFULL + s), 1);
       mbar_init(bar(BAR_VEMPTY + s), 1);
     }
@@ -128,7 +139,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 128, tDQ = tmem + 256;
+  const uint32_t tS = tmem, tP = tmem + 128, tDQ = tmem + 256, tDS = tmem + 384;
 
   if (warp == kDqProducerWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -139,29 +150,28 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tma_load_3d(sQ + b * kBox, &tmQ, b * 64, qrow0, z, bar(BAR_Q));
         tma_load_3d(sDO + b * kBox, &tmDO, b * 64, qrow0, z, bar(BAR_Q));
       }
-      int nK[kStages] = {0, 0}, nV[kStages] = {0, 0};
+      int nK[kKStages] = {0, 0, 0}, nV[kVStages] = {0, 0};
       const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool) -> bool {
-        const int s = j & 1;
-        const uint32_t ph = (uint32_t)((j >> 1) & 1);
+        const int ks = j % kKStages, vs = j & 1;
         const int krow = t * g.N + ch * kChunk;
-        if (!wait_bounded(bar(BAR_KEMPTY + s), ph ^ 1u, ctl)) return false;
-        mbar_expect_tx(bar(BAR_KFULL + s), kTileBytes);
-        tma_load_3d(sK + s * kTileBytes, &tmK, 0, krow, z, bar(BAR_KFULL + s));
-        tma_load_3d(sK + s * kTileBytes + kBox, &tmK, 64, krow, z, bar(BAR_KFULL + s));
-        ++nK[s];
-        if (!wait_bounded(bar(BAR_VEMPTY + s), ph ^ 1u, ctl)) return false;
-        mbar_expect_tx(bar(BAR_VFULL + s), kTileBytes);
-        tma_load_3d(sV + s * kTileBytes, &tmV, 0, krow, z, bar(BAR_VFULL + s));
-        tma_load_3d(sV + s * kTileBytes + kBox, &tmV, 64, krow, z, bar(BAR_VFULL + s));
-        ++nV[s];
+        if (!wait_bounded(bar(BAR_KEMPTY + ks), (uint32_t)(((j / kKStages) & 1) ^ 1), ctl)) return false;
+        mbar_expect_tx(bar(BAR_KFULL + ks), kTileBytes);
+        tma_load_3d(sK + ks * kTileBytes, &tmK, 0, krow, z, bar(BAR_KFULL + ks));
+        tma_load_3d(sK + ks * kTileBytes + kBox, &tmK, 64, krow, z, bar(BAR_KFULL + ks));
+        ++nK[ks];
+        if (!wait_bounded(bar(BAR_VEMPTY + vs), (uint32_t)(((j >> 1) & 1) ^ 1), ctl)) return false;
+        mbar_expect_tx(bar(BAR_VFULL + vs), kTileBytes);
+        tma_load_3d(sV + vs * kTileBytes, &tmV, 0, krow, z, bar(BAR_VFULL + vs));
+        tma_load_3d(sV + vs * kTileBytes + kBox, &tmV, 64, krow, z, bar(BAR_VFULL + vs));
+        ++nV[vs];
         return true;
       });
       if (n < 0) {
         drain_wait(bar(BAR_Q), 0, kTimeoutNs);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s)
           if (nK[s] > 0) drain_wait(bar(BAR_KFULL + s), (uint32_t)((nK[s] - 1) & 1), kTimeoutNs);
+        for (int s = 0; s < kVStages; ++s)
           if (nV[s] > 0) drain_wait(bar(BAR_VFULL + s), (uint32_t)((nV[s] - 1) & 1), kTimeoutNs);
-        }
       }
     }
   } else if (warp == kDqMmaWarp) {
@@ -171,45 +181,42 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // in shared memory, so S and dP of the next chunk run during this chunk's exponentials.
     if (lane == 0) {
       const bool ok = wait_bounded(bar(BAR_Q), 0, ctl);
-      // dQ += dS(jp) K(jp): A = dS (K-major in shared memory), B = K stage read MN-major
+      // dQ += dS(jp) K(jp): A = dS in tensor memory, B = K stage read MN-major
       auto dq_step = [&](int jp) -> bool {
         if (!wait_bounded(bar(BAR_DSREADY), (uint32_t)(jp & 1), ctl)) return false;
         tc_fence_after();
-        const uint32_t kb = sK + (jp & 1) * kTileBytes;
+        const uint32_t kb = sK + (jp % kKStages) * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
-          mma_ss(tDQ, desc_kmajor(sDS + off), desc_mnmajor(kb + 2048u * kk), kIdescKMN, (jp > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDQ, tDS + pcol(kk), desc_mnmajor(kb + 2048u * kk), kIdescKMN, (jp > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(BAR_DQDONE));
-        tc_commit(bar(BAR_KEMPTY + (jp & 1)));
+        tc_commit(bar(BAR_KEMPTY + jp % kKStages));
         return true;
       };
       int n = -1;
       if (ok) {
         n = for_each_chunk(g, tb, list, cnt, [&](int j, int, int, bool) -> bool {
-          const int s = j & 1;
-          const uint32_t ph = (uint32_t)((j >> 1) & 1);
+          const int ks = j % kKStages, vs = j & 1;
           if (j > 0) {
             if (!wait_bounded(bar(BAR_SFREE), (uint32_t)((j - 1) & 1), ctl)) return false;
             tc_fence_after();
           }
-          if (!wait_bounded(bar(BAR_KFULL + s), ph, ctl)) return false;
+          if (!wait_bounded(bar(BAR_KFULL + ks), (uint32_t)((j / kKStages) & 1), ctl)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tS, desc_kmajor(sQ + off), desc_kmajor(sK + s * kTileBytes + off), kIdescKK, kk > 0 ? 1u : 0u);
+            mma_ss(tS, desc_kmajor(sQ + off), desc_kmajor(sK + ks * kTileBytes + off), kIdescKK, kk > 0 ? 1u : 0u);
           }
-          if (!wait_bounded(bar(BAR_VFULL + s), ph, ctl)) return false;
+          if (!wait_bounded(bar(BAR_VFULL + vs), (uint32_t)((j >> 1) & 1), ctl)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (uint32_t)(kk >> 2) * kBox + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tP, desc_kmajor(sDO + off), desc_kmajor(sV + s * kTileBytes + off), kIdescKK, kk > 0 ? 1u : 0u);
+            mma_ss(tP, desc_kmajor(sDO + off), desc_kmajor(sV + vs * kTileBytes + off), kIdescKK, kk > 0 ? 1u : 0u);
           }
           tc_commit(bar(BAR_SFULL));
-          tc_commit(bar(BAR_VEMPTY + s));
+          tc_commit(bar(BAR_VEMPTY + vs));
           return j == 0 ? true : dq_step(j - 1);
         });
       }
@@ -234,7 +241,6 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint64_t c2 = f2_pack(scale_log2, scale_log2);
     const float nl = live ? -L2 : -INFINITY;
     const uint64_t nl2 = f2_pack(nl, nl), nd2 = f2_pack(-Dr, -Dr);
-    uint8_t* ds_row = base_ptr + kOffDS + half * kBox + r * 128;   // this thread's 64 keys: one box row
     const int n = for_each_chunk(g, tb, list, cnt, [&](int j, int t, int ch, bool full) -> bool {
       if (!wait_warp(bar(BAR_SFULL), (uint32_t)(j & 1), ctl)) return false;
       tc_fence_after();
@@ -263,14 +269,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(dpv[2 * i], dpv[2 * i + 1]), nd2)), ds0, ds1);
         pk[i] = pack_bf16x2(ds0, ds1);
       }
-      // dQ(j-1) reads dS from shared memory: it must have finished before dS is overwritten
+      // dQ(j-1) reads dS from tensor memory: it must have finished before dS is overwritten
       if (j > 0 && !wait_warp(bar(BAR_DQDONE), (uint32_t)((j - 1) & 1), ctl)) return false;
-      // 16-byte chunk c of the row (keys 8c..8c+7 of this half) at position c ^ (r mod 8)
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(ds_row + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor cores
+      tc_fence_after();
+      tmem_st32u(tDS + lane_off + 64u * half, pk);
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(bar(BAR_DSREADY));
       return true;
     });
@@ -401,13 +405,6 @@ enum : int {
   KB_KV = 0, KB_QFULL = 1, KB_QEMPTY = 4, KB_OFULL = 7, KB_OEMPTY = 9, KB_SFULL = 11, KB_PREADY = 12,
   KB_DPFULL = 13, KB_DSREADY = 14, KB_DONE = 15, KB_DRAIN = 16
 };
-
-// P^T and dS^T are written back in bf16 pairs over the fp32 columns each warp read:
-// query columns 64h .. 64h+63 of S^T (or dP^T) hold, packed, in tensor-memory
-// columns 64h .. 64h+31.  (Packing both halves into columns 0 .. 63 would let the
-// warp of half 1 overwrite fp32 values the warp of half 0 has not loaded yet.)
-// Column of the bf16 A operand for query columns 16 kk .. 16 kk + 15:
-__device__ __forceinline__ uint32_t pcol(int kk) { return 8u * (uint32_t)kk + ((uint32_t)(kk >> 2) << 5); }
 
 // Calls f(step, t, ch) for every 128-row chunk with a valid row of every query tile
 // in the transposed list, in list order; stops early when f returns false.

@@ -8,9 +8,9 @@
 // no part (dQ = 0) and pad keys get dK = dV = 0.
 //
 // Kernels, in launch order:
-//   bwd_rowdot_kernel     D per packed row (one warp per row); for bf16 also
-//                         -LSE * log2(e) and -D per row of whole tiles, as the
-//                         tensor-core dK/dV kernel reads them.
+//   bwd_rowdot_kernel     D per packed row (fp32; bf16 runs bwd_rowstat_tc_kernel,
+//                         which also writes -LSE * log2(e) and -D per row of whole
+//                         tiles, as the tensor-core dK/dV kernel reads them).
 //   bwd_transpose_kernel  for each key tile, the ascending list of query tiles
 //                         that keep it (one warp per key tile: a binary search
 //                         in every query tile's sorted list, ballots, prefix).
@@ -24,6 +24,8 @@
 #include "ssta_internal.h"
 
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 namespace ssta {
 namespace {
@@ -88,31 +90,33 @@ __device__ __forceinline__ bool row_valid(const Geom& g, int t, const TileValid&
   return o < v.text;
 }
 
+// D = rowsum(dO * O) per packed row for the fp32 kernels (bf16 uses
+// bwd_rowstat_tc_kernel): each lane reads 16 bytes (4 channels), 32 lanes per row,
+// four rows per warp with every load issued before the first sum; grid.y is the head.
+constexpr int kRowdotRows = 4;
 template <typename T>
 __global__ void __launch_bounds__(kBwdWarps * 32)
-bwd_rowdot_kernel(Geom g, const T* __restrict__ o, const T* __restrict__ dO, const float* __restrict__ lse,
-                  float* __restrict__ Dv, float* __restrict__ nl2, float* __restrict__ nd) {
+bwd_rowdot_kernel(Geom g, int64_t bh0, const T* __restrict__ o, const T* __restrict__ dO, float* __restrict__ Dv) {
   const int lane = threadIdx.x & 31;
-  const int64_t Lp = (int64_t)g.NQ * g.N;   // whole tiles: the last text tile's tail rows too
-  const int64_t w = (int64_t)blockIdx.x * kBwdWarps + (threadIdx.x >> 5);   // bh * Lp + row
-  if (w >= (int64_t)g.B * g.H * Lp) return;
-  const int64_t bh = w / Lp, row = w - bh * Lp;
-  const int t = (int)(row / g.N);
-  const bool valid = row < g.Lq && row_valid(g, t, tile_valid(g, t), (int)(row - (int64_t)t * g.N));
-  const int64_t wq = bh * g.Lq + row;
-  float d = 0.f, unused = 0.f;
-  if (valid) {
-    d = dot4(load4(o, wq, lane), load4(dO, wq, lane));
-    warp_sum2(d, unused);
+  const int64_t bh = bh0 + blockIdx.y;
+  const int64_t r0 = ((int64_t)blockIdx.x * kBwdWarps + (threadIdx.x >> 5)) * kRowdotRows;
+  float4 va[kRowdotRows], vb[kRowdotRows];
+  bool valid[kRowdotRows];
+#pragma unroll
+  for (int it = 0; it < kRowdotRows; ++it) {
+    const int64_t row = r0 + it;
+    const int t = (int)(row / g.N);
+    valid[it] = row < g.Lq && row_valid(g, t, tile_valid(g, t), (int)(row - (int64_t)t * g.N));
+    va[it] = valid[it] ? load4(o, bh * g.Lq + row, lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+    vb[it] = valid[it] ? load4(dO, bh * g.Lq + row, lane) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (lane == 0) {
-    if (row < g.Lq) Dv[wq] = d;
-    if (nl2 != nullptr) {
-      // the tensor-core dK/dV kernel adds these: -LSE in log2 units (-inf for a row that
-      // takes no part, whose P is then exactly 0) and -D
-      const float L = valid ? lse[wq] : -INFINITY;
-      nl2[w] = L > -INFINITY ? -(L * 1.4426950408889634f) : -INFINITY;
-      nd[w] = L > -INFINITY ? -d : 0.f;
+#pragma unroll
+  for (int it = 0; it < kRowdotRows; it += 2) {
+    float d0 = dot4(va[it], vb[it]), d1 = dot4(va[it + 1], vb[it + 1]);
+    warp_sum2(d0, d1);
+    if (lane == 0) {
+      if (r0 + it < g.Lq) Dv[bh * g.Lq + r0 + it] = d0;
+      if (r0 + it + 1 < g.Lq) Dv[bh * g.Lq + r0 + it + 1] = d1;
     }
   }
 }
@@ -249,9 +253,6 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
                              void* dq, void* dk, void* dv, const BwdWorkspace& ws, uint8_t* base, cudaStream_t s) {
   const int64_t rows = (int64_t)g.B * g.H * g.Lq, tiles = (int64_t)g.B * g.H * g.NQ;
   float* Dv = reinterpret_cast<float*>(base + ws.rowdot);
-  float* nl2 = kTensorCores<T> ? reinterpret_cast<float*>(base + ws.nl2) : nullptr;
-  float* nd = kTensorCores<T> ? reinterpret_cast<float*>(base + ws.nd) : nullptr;
-  const int64_t prows = (int64_t)g.B * g.H * g.NQ * g.N;
   int32_t* tidx = reinterpret_cast<int32_t*>(base + ws.tidx);
   int32_t* tcnt = reinterpret_cast<int32_t*>(base + ws.tcnt);
   int32_t* status = reinterpret_cast<int32_t*>(base + ws.status);
@@ -260,8 +261,18 @@ cudaError_t launch_bwd_typed(const Geom& g, const void* q, const void* k, const 
   const T* tk = static_cast<const T*>(k);
   const T* tv = static_cast<const T*>(v);
   const T* tO = static_cast<const T*>(dO);
-  const unsigned pb = (unsigned)((prows + kBwdWarps - 1) / kBwdWarps);
-  bwd_rowdot_kernel<T><<<pb, kBwdWarps * 32, 0, s>>>(g, static_cast<const T*>(o), tO, lse, Dv, nl2, nd);
+  float* nl2 = reinterpret_cast<float*>(base + ws.nl2);
+  float* nd = reinterpret_cast<float*>(base + ws.nd);
+  if constexpr (kTensorCores<T>) {
+    cudaError_t e = launch_attention_bwd_rowstat_tc(g, o, dO, lse, Dv, nl2, nd, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    const int64_t rows_per_block = (int64_t)kBwdWarps * kRowdotRows, BH = (int64_t)g.B * g.H;
+    for (int64_t bh0 = 0; bh0 < BH; bh0 += 65535) {   // grid.y holds at most 65535 heads
+      const dim3 grid((unsigned)((g.Lq + rows_per_block - 1) / rows_per_block), (unsigned)std::min<int64_t>(BH - bh0, 65535));
+      bwd_rowdot_kernel<T><<<grid, kBwdWarps * 32, 0, s>>>(g, bh0, static_cast<const T*>(o), tO, Dv);
+    }
+  }
   bwd_transpose_kernel<<<tb, kBwdWarps * 32, 0, s>>>(g, kv_idx, kv_cnt, tidx, tcnt, status);
   if constexpr (kTensorCores<T>) {   // bf16: the API guarantees N % 128 == 0
     cudaError_t e = launch_attention_bwd_dq_tc(g, q, k, v, dO, lse, Dv, kv_idx, kv_cnt, dq, status, s);

@@ -23,6 +23,8 @@
 // Every wait is bounded (ssta_wait.cuh), as in the forward kernel.
 #include "ssta_tc_common.cuh"
 
+#include <algorithm>
+
 namespace ssta {
 namespace {
 
@@ -321,6 +323,80 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 }
 
 }  // namespace
+
+namespace {
+
+// Row statistics for the tensor-core kernels, per packed row of whole tiles:
+// D = rowsum(dO * O) (rows < Lq), and the values the dK/dV kernel adds,
+// -LSE * log2(e) and -D (-inf and 0 for pad rows and rows without a kept key).
+// 16 lanes per row (16-byte loads of 8 bf16 channels), 8 rows per warp with every
+// load issued before the first sum; row validity from the tile tables, so no lane
+// divides by the grid extents; grid.y is the head.
+constexpr int kRsWarps = 8;
+constexpr int kRsRows = 8;   // rows per warp
+
+__global__ void __launch_bounds__(kRsWarps * 32)
+bwd_rowstat_tc_kernel(const Geom g, const __grid_constant__ ChunkTables tb, int64_t bh0,
+                      const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                      const float* __restrict__ lse, float* __restrict__ Dv, float* __restrict__ nl2,
+                      float* __restrict__ nd) {
+  const int lane = threadIdx.x & 31, sub = lane >> 4, part = lane & 15;
+  const int64_t bh = bh0 + blockIdx.y;
+  const int64_t Lp = (int64_t)g.NQ * g.N;
+  const int64_t r0 = ((int64_t)blockIdx.x * kRsWarps + (threadIdx.x >> 5)) * kRsRows;
+  int4 va[kRsRows / 2], vb[kRsRows / 2];
+  bool valid[kRsRows / 2];
+#pragma unroll
+  for (int it = 0; it < kRsRows / 2; ++it) {
+    const int64_t row = r0 + 2 * it + sub;
+    bool ok = row < g.Lq;   // rows past Lq exist only in the last text tile
+    if (ok) {
+      const int t = (int)(row / g.N);
+      ok = key_valid(g, tb, t, (int)(row - (int64_t)t * g.N));
+    }
+    valid[it] = ok;
+    const int64_t wq = bh * g.Lq + row;
+    va[it] = ok ? reinterpret_cast<const int4*>(o + wq * 128)[part] : make_int4(0, 0, 0, 0);
+    vb[it] = ok ? reinterpret_cast<const int4*>(dO + wq * 128)[part] : make_int4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int it = 0; it < kRsRows / 2; ++it) {
+    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&va[it]);
+    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&vb[it]);
+    float d = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+      d = fmaf(u.x, v.x, d);
+      d = fmaf(u.y, v.y, d);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    const int64_t row = r0 + 2 * it + sub;
+    if (part == 0 && row < Lp) {
+      const int64_t wq = bh * g.Lq + row;
+      if (row < g.Lq) Dv[wq] = d;
+      const float L = valid[it] ? lse[wq] : -INFINITY;
+      nl2[bh * Lp + row] = L > -INFINITY ? -(L * 1.4426950408889634f) : -INFINITY;
+      nd[bh * Lp + row] = L > -INFINITY ? -d : 0.f;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention_bwd_rowstat_tc(const Geom& g, const void* o, const void* dO, const float* lse, float* Dv,
+                                            float* nl2, float* nd, cudaStream_t s) {
+  const int64_t BH = (int64_t)g.B * g.H;
+  const int64_t Lp = (int64_t)g.NQ * g.N, rows_per_block = (int64_t)kRsWarps * kRsRows;
+  const ChunkTables tb = make_chunk_tables(g);
+  for (int64_t bh0 = 0; bh0 < BH; bh0 += 65535) {   // grid.y holds at most 65535 heads
+    const dim3 grid((unsigned)((Lp + rows_per_block - 1) / rows_per_block), (unsigned)std::min<int64_t>(BH - bh0, 65535));
+    bwd_rowstat_tc_kernel<<<grid, kRsWarps * 32, 0, s>>>(g, tb, bh0, static_cast<const __nv_bfloat16*>(o),
+                                                         static_cast<const __nv_bfloat16*>(dO), lse, Dv, nl2, nd);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
                                        const float* lse, const float* Dv, const int32_t* kv_idx,

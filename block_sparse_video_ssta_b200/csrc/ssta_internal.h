@@ -100,6 +100,8 @@ cudaError_t launch_attention_bwd_dq_tc(const Geom& g, const void* q, const void*
                                        const float* lse, const float* Dv, const int32_t* kv_idx,
                                        const int32_t* kv_cnt, void* dq, int32_t* status, cudaStream_t s);
 // bf16, N % 128 == 0: dK and dV on the tensor cores (tidx/tcnt: the transposed lists).
+cudaError_t launch_attention_bwd_rowstat_tc(const Geom& g, const void* o, const void* dO, const float* lse, float* Dv,
+                                            float* nl2, float* nd, cudaStream_t s);
 cudaError_t launch_attention_bwd_dkdv_tc(const Geom& g, const void* q, const void* k, const void* v, const void* dO,
                                          const float* nl2, const float* nd, const int32_t* tidx,
                                          const int32_t* tcnt, void* dk, void* dv, int32_t* status, cudaStream_t s);

@@ -189,7 +189,7 @@ ssta_status ssta_build_block_mask(const ssta_desc* desc, const void* q_packed, c
   // the pool kernel also clears the status word
   cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, reinterpret_cast<int32_t*>(w + ws.status), ib, s);
   if (e == cudaSuccess && imp) e = launch_tile_keysum(g, kbar, ib, s);
-  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
+  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, reinterpret_cast<int32_t*>(w + ws.status), s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return from_cuda(e);
 }

@@ -84,9 +84,12 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
                              int32_t* status, const ImportanceBufs& ib, cudaStream_t s);
 // Importance score only: per 32-tile block sums of the unit key means.
 cudaError_t launch_tile_keysum(const Geom& g, const float* kbar, const ImportanceBufs& ib, cudaStream_t s);
-// Block scores: raw dot products, or the importance score when ib.ksum != NULL.
+// Block scores: raw dot products (on the tensor cores, ssta_mask_tc.cu), or the
+// importance score when ib.ksum != NULL (SIMT).  `status` may be NULL.
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
-                               float* scores, cudaStream_t s);
+                               float* scores, int32_t* status, cudaStream_t s);
+cudaError_t launch_tile_scores_tc(const Geom& g, const float* qbar, const float* kbar, float* scores,
+                                  int32_t* status, cudaStream_t s);
 cudaError_t launch_select_and_list(const Geom& g, const float* scores, int32_t* kv_idx, int32_t* kv_cnt,
                                    cudaStream_t s);
 cudaError_t launch_attention_f32(const Geom& g, const float* qp, const float* kp, const float* vp,

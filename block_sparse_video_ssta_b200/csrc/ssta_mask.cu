@@ -16,11 +16,14 @@
 //                         the score kernel turns them into each key tile's
 //                         redundancy (mean key-key similarity to the other key
 //                         tiles) in O(NT*D) per head, without an NT x NT product.
-//   tile_scores_kernel    fp32 SIMT, 128x128 score blocks per CTA, 8x8 per
-//                         thread, 16-channel stages double-buffered in shared
-//                         memory by cp.async, channels summed in order 0..D-1
-//                         with FMA (packed f32x2, two columns per instruction);
-//                         the importance score is formed in the epilogue.
+//   tile_scores_tc_kernel similarity score on the tensor cores, fp32 means split
+//                         into three bf16 parts (ssta_mask_tc.cu).
+//   tile_scores_kernel    importance score: fp32 SIMT, 128x128 score blocks per CTA,
+//                         8x8 per thread, 16-channel stages double-buffered in
+//                         shared memory by cp.async, channels summed in order
+//                         0..D-1 with FMA (packed f32x2, two columns per
+//                         instruction); the importance score is formed in the
+//                         epilogue.
 //   select_and_list_kernel one warp per (head, query tile): top-k over scores
 //                         held in registers as order-preserving 32-bit keys
 //                         (bitwise binary search for the k-th key with warp-wide
@@ -632,8 +635,9 @@ cudaError_t launch_tile_keysum(const Geom& g, const float* kbar, const Importanc
 }
 
 cudaError_t launch_tile_scores(const Geom& g, const float* qbar, const float* kbar, const ImportanceBufs& ib,
-                               float* scores, cudaStream_t s) {
+                               float* scores, int32_t* status, cudaStream_t s) {
   if ((int64_t)g.B * g.H == 0) return cudaSuccess;
+  if (ib.ksum == nullptr) return launch_tile_scores_tc(g, qbar, kbar, scores, status, s);
   dim3 grid(ceil_div(g.NT, kScoreBlock), ceil_div(g.NT, kScoreBlock), g.B * g.H);
   if (g.NT % 4 == 0)
     return launch_dependent(tile_scores_kernel<true>, grid, dim3(256), 0, s, g, qbar, kbar, ib, scores);

@@ -90,7 +90,7 @@ extern "C" ssta_status ssta_build_block_mask_noalloc(const ssta_desc* desc, cons
   // no status word (nullptr): nothing could read it back
   cudaError_t e = launch_tile_pool(g, q_packed, k_packed, qbar, kbar, nullptr, ib, s);
   if (e == cudaSuccess && imp) e = launch_tile_keysum(g, kbar, ib, s);
-  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, s);
+  if (e == cudaSuccess) e = launch_tile_scores(g, qbar, kbar, ib, scores, nullptr, s);
   if (e == cudaSuccess) e = launch_select_and_list(g, scores, kv_idx, kv_cnt, s);
   return from_cuda(e);
 }

@@ -412,7 +412,7 @@ constexpr int kHiBits = 12;       // prefix bits searched over every key
 constexpr int kHiBitsWide = 16;   // ... when the 12-bit bucket holds more than kBucketCap keys
 
 template <int SLOTS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)   // 4 CTAs per SM: 62 registers, no spills at SLOTS <= 32
 select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __restrict__ kv_idx,
                        int32_t* __restrict__ kv_cnt) {
   __shared__ uint32_t bucket_smem[8 * kBucketCap];

@@ -89,27 +89,50 @@ tile_scores_tc_kernel(const Geom g, const float* __restrict__ qbar_t, const floa
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
 
-  bool ok = true;
-  uint32_t tmem = 0;
-  int issued = 0;   // passes whose MMAs thread 0 committed
-  for (int pass = 0; pass < 2 && ok; ++pass) {
-    // ---- 1. split the means of channels 64 pass .. +63.  Item = (operand, channel, group
-    // of 8 tiles): 2 x 64 x 16 items, 8 per thread; consecutive threads take consecutive
-    // groups of one channel, so each warp reads two 512-byte channel rows.
+  // every load of a pass is issued before the first is used: vector loads (predicated, no
+  // branch) for groups of 8 tiles inside NT, then scalar loads for a ragged or unaligned
+  // group.  Item = (operand, channel, group of 8 tiles): 2 x 64 x 16 items per pass, 8 per
+  // thread; consecutive threads take consecutive groups of one channel, so each warp reads
+  // two 512-byte channel rows.
+  float4 va[8], vb[8];
+  auto load_pass = [&](int pass) {
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int item = (int)threadIdx.x + kScThreads * r;
       const int g8 = item & 15, ch = (item >> 4) & 63, op = item >> 10;
       const int t0 = (op ? j0 : i0) + 8 * g8;
-      const float* src = (op ? kbar_t : qbar_t) + (bh * g.D + kScChannels * pass + ch) * (int64_t)NT + t0;
-      float v[8];
-      if (vec && t0 + 8 <= NT) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-      } else {
+      const float4* src = reinterpret_cast<const float4*>((op ? kbar_t : qbar_t) +
+                                                          (bh * g.D + kScChannels * pass + ch) * (int64_t)NT + t0);
+      const bool full = vec && t0 + 8 <= NT;
+      va[r] = full ? __ldg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+      vb[r] = full ? __ldg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = t0 + e < NT ? __ldg(src + e) : 0.f;
+    for (int r = 0; r < 8; ++r) {
+      const int item = (int)threadIdx.x + kScThreads * r;
+      const int g8 = item & 15, ch = (item >> 4) & 63, op = item >> 10;
+      const int t0 = (op ? j0 : i0) + 8 * g8;
+      if (!(vec && t0 + 8 <= NT) && t0 < NT) {
+        const float* src = (op ? kbar_t : qbar_t) + (bh * g.D + kScChannels * pass + ch) * (int64_t)NT + t0;
+        float w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = t0 + e < NT ? __ldg(src + e) : 0.f;
+        va[r] = make_float4(w[0], w[1], w[2], w[3]);
+        vb[r] = make_float4(w[4], w[5], w[6], w[7]);
       }
+    }
+  };
+
+  bool ok = true;
+  int issued = 0;   // passes whose MMAs thread 0 committed
+  load_pass(0);
+  for (int pass = 0; pass < 2 && ok; ++pass) {
+    // ---- 1. split the loaded means of channels 64 pass .. +63 into the operand layout
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int item = (int)threadIdx.x + kScThreads * r;
+      const int g8 = item & 15, ch = (item >> 4) & 63, op = item >> 10;
+      const float v[8] = {va[r].x, va[r].y, va[r].z, va[r].w, vb[r].x, vb[r].y, vb[r].z, vb[r].w};
       __align__(16) __nv_bfloat16 hp[8], mp[8], lp[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) split3(v[e], hp[e], mp[e], lp[e]);
@@ -125,7 +148,7 @@ tile_scores_tc_kernel(const Geom g, const float* __restrict__ qbar_t, const floa
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    tmem = *tmem_slot;
+    const uint32_t tmem = *tmem_slot;
 
     // ---- 2. the six products, smallest first, into one accumulator
     if (threadIdx.x == 0) {
@@ -142,10 +165,12 @@ tile_scores_tc_kernel(const Geom g, const float* __restrict__ qbar_t, const floa
       ++issued;
     }
     __syncwarp();
-    ok = wait_warp(bar, (uint32_t)pass, ctl);   // the operands are read before they are overwritten
+    if (pass == 0) load_pass(1);                  // in flight while the tensor cores work
+    ok = wait_warp(bar, (uint32_t)pass, ctl);     // the operands are read before they are overwritten
     ok = __syncthreads_and(ok);
     tc_fence_after();
   }
+  const uint32_t tmem = *tmem_slot;
 
   // ---- 3. scores out: warp w holds query tile i0 + 32 (w mod 4) + lane, key tiles
   // j0 + 64 (w / 4) .. +63

@@ -24,9 +24,12 @@
  *  - Errors: arguments are checked on the host before anything is launched.
  *    Launch failures return SSTA_ERR_LAUNCH.  Faults the kernels detect on the
  *    device (an out-of-range kept-tile id, a pipeline wait that exceeded its
- *    time limit) do not trap: the kernel records a code in the first 4 bytes
- *    of the workspace (an int32; 0 = no error, else an ssta_status value) and
- *    returns; read it with ssta_read_device_status after the stream completes.
+ *    time limit, or - in the backward dK/dV kernel, whose shared-memory layout
+ *    leaves under 1 KB to align its base - a dynamic shared-memory base the
+ *    runtime did not place 1024-byte aligned, SSTA_ERR_ALIGNMENT) do not trap:
+ *    the kernel records a code in the first 4 bytes of the workspace (an int32;
+ *    0 = no error, else an ssta_status value) and returns; read it with
+ *    ssta_read_device_status after the stream completes.
  *  - Calls are stateless and thread-safe; separate calls may run concurrently
  *    on different streams if their workspaces differ.
  *  - Dtypes: SSTA_BF16 (bfloat16 storage; tensor-core attention with fp32

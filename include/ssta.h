@@ -154,7 +154,9 @@ ssta_status ssta_tile_reorder(const ssta_desc* desc, const void* x_raster, const
 /*
  * ssta_build_block_mask — Steps 2-4 up to the mask: per (b, h, video tile) mean
  * of q and k over the tile's valid tokens; fp32 block scores (Step 2: Score_s =
- * Qbar Kbar^T, or the importance score of desc->score_mode); per query tile the
+ * Qbar Kbar^T, computed on the tensor cores with each fp32 mean split into three
+ * bf16 parts and six products accumulated in fp32, or the importance score of
+ * desc->score_mode, computed with fp32 FMA); per query tile the
  * top-k key tiles by score, ties to the lower tile index (Step 2,
  * Topk/Indexes2mask); combined (desc->combine: union, or AND) with the sliding
  * tile window (Step 3; desc->window_mode: slid inward at the grid edges so it

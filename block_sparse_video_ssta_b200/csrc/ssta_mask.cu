@@ -83,11 +83,33 @@ __device__ __forceinline__ void add_vec(float* acc, const int4& raw, const float
   for (int i = 0; i < 4; ++i) acc[i] += f[i];
 }
 
+// Valid rows of a video tile, one bit per token, for each of the 8 tile classes (bit 2 of
+// the class: last tile along T with padding, bit 1: along Y, bit 0: along X); built on the
+// host, so a partial tile's rows are tested with a shift instead of three divisions.
+constexpr int kMaxRowWords = 4096 / 32;   // N <= 4096
+struct PoolRowMask {
+  uint32_t w[8][kMaxRowWords];
+};
+PoolRowMask make_pool_row_mask(const Geom& g) {
+  PoolRowMask m{};
+  for (int cls = 0; cls < 8; ++cls) {
+    const int vt = (cls & 4) ? g.T - (g.nT - 1) * g.tT : g.tT;
+    const int vy = (cls & 2) ? g.Y - (g.nY - 1) * g.tY : g.tY;
+    const int vx = (cls & 1) ? g.X - (g.nX - 1) * g.tX : g.tX;
+    for (int o = 0; o < g.N && o < 32 * kMaxRowWords; ++o) {
+      const int dx = o % g.tX, dy = (o / g.tX) % g.tY, dt = o / (g.tX * g.tY);
+      if (dt < vt && dy < vy && dx < vx) m.w[cls][o >> 5] |= 1u << (o & 31);
+    }
+  }
+  return m;
+}
+
 // Step 2, pooled (average) representation of each video tile over its valid tokens.
 template <typename T>
-__global__ void __launch_bounds__(kPoolThreads)
-tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ kp,
-                 float* __restrict__ qbar, float* __restrict__ kbar, int32_t* __restrict__ status, ImportanceBufs ib) {
+__global__ void __launch_bounds__(kPoolThreads, 4)   // 64 registers: four CTAs per SM
+tile_pool_kernel(Geom g, const __grid_constant__ PoolRowMask rm, const int4* __restrict__ qp,
+                 const int4* __restrict__ kp, float* __restrict__ qbar, float* __restrict__ kbar,
+                 int32_t* __restrict__ status, ImportanceBufs ib) {
   allow_dependents();
   grid_dependency_wait();   // q and k are packed by the previous kernels
   if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
@@ -103,6 +125,12 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
   const int vt = axis_valid(cT, g.tT, g.T), vy = axis_valid(cY, g.tY, g.Y),
             vx = axis_valid(cX, g.tX, g.X);
   const bool full = (vt == g.tT) && (vy == g.tY) && (vx == g.tX);
+  __shared__ uint32_t mask[kMaxRowWords];   // this tile's valid rows (partial tiles)
+  if (!full) {
+    const int cls = (vt < g.tT ? 4 : 0) | (vy < g.tY ? 2 : 0) | (vx < g.tX ? 1 : 0);
+    for (int i = threadIdx.x; i < (g.N + 31) / 32; i += kPoolThreads) mask[i] = rm.w[cls][i];
+    __syncthreads();
+  }
 
   const int64_t base = (bh * g.Lq + (int64_t)c * g.N) * vpr + vec;
   float aq[EPV], ak[EPV];
@@ -129,9 +157,27 @@ tile_pool_kernel(Geom g, const int4* __restrict__ qp, const int4* __restrict__ k
       add_vec(ak, __ldg(kp + base + (int64_t)o * vpr), (const T*)nullptr);
     }
   } else {
-    for (int o = rsub; o < g.N; o += rpp) {
-      const int dx = o % g.tX, dy = (o / g.tX) % g.tY, dt = o / (g.tX * g.tY);
-      if (dt < vt && dy < vy && dx < vx) {
+    // the same batched loads; pad rows load nothing and add zeros, which leaves every sum
+    // (taken in the same row order) unchanged
+    const int4 zero = make_int4(0, 0, 0, 0);
+    int o = rsub;
+    for (; o + 7 * rpp < g.N; o += 8 * rpp) {
+      int4 rq[8], rk[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = o + u * rpp;
+        const bool ok = (mask[r >> 5] >> (r & 31)) & 1u;
+        rq[u] = ok ? __ldg(qp + base + (int64_t)r * vpr) : zero;
+        rk[u] = ok ? __ldg(kp + base + (int64_t)r * vpr) : zero;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        add_vec(aq, rq[u], (const T*)nullptr);
+        add_vec(ak, rk[u], (const T*)nullptr);
+      }
+    }
+    for (; o < g.N; o += rpp) {
+      if ((mask[o >> 5] >> (o & 31)) & 1u) {
         add_vec(aq, __ldg(qp + base + (int64_t)o * vpr), (const T*)nullptr);
         add_vec(ak, __ldg(kp + base + (int64_t)o * vpr), (const T*)nullptr);
       }
@@ -622,10 +668,11 @@ cudaError_t launch_tile_pool(const Geom& g, const void* qp, const void* kp, floa
   const size_t smem = 2 * rpp * g.D * sizeof(float);
   const int4* q4 = static_cast<const int4*>(qp);
   const int4* k4 = static_cast<const int4*>(kp);
+  const PoolRowMask rm = make_pool_row_mask(g);
   if (g.dtype == SSTA_BF16)
-    return launch_dependent(tile_pool_kernel<__nv_bfloat16>, grid, dim3(kPoolThreads), smem, s, g, q4, k4, qbar,
+    return launch_dependent(tile_pool_kernel<__nv_bfloat16>, grid, dim3(kPoolThreads), smem, s, g, rm, q4, k4, qbar,
                             kbar, status, ib);
-  return launch_dependent(tile_pool_kernel<float>, grid, dim3(kPoolThreads), smem, s, g, q4, k4, qbar, kbar,
+  return launch_dependent(tile_pool_kernel<float>, grid, dim3(kPoolThreads), smem, s, g, rm, q4, k4, qbar, kbar,
                           status, ib);
 }
 

@@ -84,6 +84,7 @@ CASES = [
     ("small_bf16", dict(H=2, T=4, Y=8, X=16, tT=2, tY=8, tX=8)),           # N = 128
     ("small_bf16", dict(H=2, T=8, Y=16, X=16, tT=4, tY=8, tX=16, L_text=40)),  # N = 512
     ("small_bf16", dict(H=2, T=8, Y=16, X=24, score_mode="importance", combine="and", topk=6, wT=3, wY=3, wX=3)),
+    ("small_bf16", dict(B=2, H=3, T=5, Y=12, X=20, L_text=130)),          # batch 2, odd heads, ragged, partial text
 ]
 
 

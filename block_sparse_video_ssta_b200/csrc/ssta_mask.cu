@@ -48,6 +48,14 @@ using namespace f32x2;
 // allow_dependents() lets the next kernel start launching.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// A pointer to data the previous kernel writes, passed through an empty asm after the wait: the
+// compiler then cannot issue loads through it (which it may treat as reads of invariant memory,
+// being const __restrict__) ahead of griddepcontrol.wait.
+template <typename T>
+__device__ __forceinline__ T* after_wait(T* p) {
+  asm volatile("" : "+l"(p)::"memory");
+  return p;
+}
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
@@ -112,6 +120,8 @@ tile_pool_kernel(Geom g, const __grid_constant__ PoolRowMask rm, const int4* __r
                  int32_t* __restrict__ status, ImportanceBufs ib) {
   allow_dependents();
   grid_dependency_wait();   // q and k are packed by the previous kernels
+  qp = after_wait(qp);
+  kp = after_wait(kp);
   if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
   constexpr int EPV = 16 / sizeof(T);        // elements per 16-byte vector
   const int vpr = g.D / EPV;                 // vectors per row
@@ -233,6 +243,8 @@ __global__ void __launch_bounds__(128)
 tile_keysum_kernel(Geom g, const float* __restrict__ kbar_t, ImportanceBufs ib) {
   allow_dependents();
   grid_dependency_wait();   // the means and norms are written by the previous kernel
+  kbar_t = after_wait(kbar_t);
+  ib.inv_nk = after_wait(ib.inv_nk);
   const int64_t bh = blockIdx.y;
   const int NT = g.NT;
   const int c0 = blockIdx.x * kKeySumTiles, c1 = min(c0 + kKeySumTiles, NT);
@@ -318,6 +330,11 @@ tile_scores_kernel(Geom g, const float* __restrict__ qbar_t, const float* __rest
   const int nst = g.D / kScoreStage;
   allow_dependents();
   grid_dependency_wait();   // the pooled means are written by the previous kernel
+  qbar_t = after_wait(qbar_t);
+  kbar_t = after_wait(kbar_t);
+  ib.inv_nq = after_wait(ib.inv_nq);
+  ib.inv_nk = after_wait(ib.inv_nk);
+  ib.ksum = after_wait(ib.ksum);
   // importance score: u = sum of the unit key means of the head (partial sums added in
   // block order), and Kbar_j . u for this CTA's 128 key tiles, accumulated from the
   // staged key means by two threads per tile (channels 0-7 and 8-15 of each stage)
@@ -466,6 +483,7 @@ select_and_list_kernel(Geom g, const float* __restrict__ scores, int32_t* __rest
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // bh * NQ + i
   if (row >= (int64_t)g.B * g.H * g.NQ) return;
   grid_dependency_wait();   // the scores are written by the previous kernel
+  scores = after_wait(scores);
   const int64_t bh = row / g.NQ;
   const int i = (int)(row - bh * g.NQ);
   int32_t* out = kv_idx + row * g.max_kept;
